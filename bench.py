@@ -1,0 +1,403 @@
+"""Benchmark of one DSA sparse-attention prefill layer on B200.
+
+A step is one pass of the whole layer (indexer scores -> exact top-k ->
+sparse attention) through dsa_prefill_layer over one synthetic chunk: by
+default the 8,192-query chunk at positions 9,216..17,407 of a 17,408-token
+context (top-2048, 32 heads, 512 + 64 latent/rope, indexer 32 x 128).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line. ``value`` is whole-job queries per second per layer
+(device time, inputs resident in HBM, L2 flushed between steps); ``e2e`` is
+the same metric through the same C-ABI call with host buffers, the
+host->device copies of the inputs and the device->host copy of the output
+inside the timed region. ``--impl reference`` times the float64 CPU oracle on
+a bounded sample of the same workload instead.
+
+Multi-GPU (torchrun): every rank runs its own chunk of the same shape (weak
+scaling, no data-path collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_LAYER = 4  # indexer scores, key-norm max, top-k, sparse attention
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------- distributed
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ our GPU path
+
+
+def run_ours(args):
+    import torch
+
+    import sparse_attention_prefill_dsa_b200 as dsa
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(local)
+    dsa.library()
+    wl = workloads.BY_NAME[args.workload]
+    d = wl.dims
+    w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
+    x = workloads.generate(d, wl.seed + 1000 * rank, wl.kind, w_mode)
+    stream = torch.cuda.current_stream()
+
+    def to_dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    xd = {k: (to_dev_bf16(v) if v.dtype == np.uint16 else torch.from_numpy(v).cuda())
+          for k, v in x.items()}
+    out = torch.empty(d.n_q, d.n_heads, d.d_latent, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(d.n_q, d.n_heads, dtype=torch.float32, device="cuda")
+    idx = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
+    ws_layer = torch.empty(dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER), dtype=torch.uint8,
+                           device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def layer():
+        dsa.check(dsa.dsa_prefill_layer(d, xd["q"], xd["latent"], xd["rope"], xd["q_idx"],
+                                        xd["k_idx"], xd["w_idx"], out, lse, idx, ws_layer,
+                                        stream=stream))
+
+    for _ in range(args.warmup):
+        layer()
+        flush.zero_()
+    dsa.check(dsa.dsa_device_status(ws_layer, stream=stream))
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps of the layer, L2 flushed (untimed) between steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for s in range(args.steps):
+            flush.zero_()
+            starts[s].record(stream)
+            layer()
+            ends[s].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    dsa.check(dsa.dsa_device_status(ws_layer, stream=stream))
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    value = world * d.n_q / (ms_per_step / 1e3)
+
+    # ---- per-kernel durations, same inputs and launch configuration
+    ld = (d.ctx_len + 127) // 128 * 128
+    scores = ws_layer[256:256 + d.n_q * ld * 4].view(torch.float32).view(d.n_q, ld)
+    ws_small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    names = ("index_scores", "topk_select", "sparse_attn")
+    ev = {n: [] for n in names}
+    for s in range(args.steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        dsa.check(dsa.dsa_index_scores(d, xd["q_idx"], xd["k_idx"], xd["w_idx"], scores, ld,
+                                       ws_small, stream=stream))
+        e[1].record(stream)
+        dsa.check(dsa.dsa_topk_select(d, scores, ld, xd["q_idx"], xd["k_idx"], xd["w_idx"], idx,
+                                      ws_small, stream=stream))
+        e[2].record(stream)
+        dsa.check(dsa.dsa_sparse_attn_prefill(d, xd["q"], xd["latent"], xd["rope"], idx, out,
+                                              lse, ws_small, stream=stream))
+        e[3].record(stream)
+        ev["index_scores"].append(e)
+    torch.cuda.synchronize()
+    per_kernel = {n: 0.0 for n in names}
+    for e in ev["index_scores"]:
+        per_kernel["index_scores"] += e[0].elapsed_time(e[1]) / args.steps
+        per_kernel["topk_select"] += e[1].elapsed_time(e[2]) / args.steps
+        per_kernel["sparse_attn"] += e[2].elapsed_time(e[3]) / args.steps
+
+    # ---- end to end through the same call with host buffers
+    pinned = {k: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
+                  if v.dtype == np.uint16 else torch.from_numpy(v)).pin_memory()
+              for k, v in x.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, t in pinned.items():
+            xd[k].copy_(t, non_blocking=True)
+        layer()
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    barrier(world)
+
+    fl = workloads.useful_flops(d)
+    peaks, peaks_src = load_peaks()
+    tflops = fl["total"] * world / (ms_per_step / 1e3) / 1e12 / world
+    dom_name = max(per_kernel, key=per_kernel.get)
+    dom_flops = {"index_scores": fl["indexer"], "sparse_attn": fl["attention"]}
+    if dom_name in dom_flops:
+        ach = dom_flops[dom_name] / (per_kernel[dom_name] / 1e3) / 1e12
+        roof = {"kernel": dom_name, "bound": "tensor", "achieved": ach,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peaks_src} bf16 burst (kernel timed alone)"}
+    else:  # top-k reads the score rows once
+        t = d.q_pos0 + np.arange(d.n_q)
+        nbytes = float(((t + 1) * 4).sum() + d.n_q * d.top_k * 4)
+        ach = nbytes / (per_kernel[dom_name] / 1e3) / 1e9
+        roof = {"kernel": dom_name, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peaks_src} copy bandwidth"}
+
+    result = {
+        "metric": "DSA prefill queries/s per layer",
+        "value": value,
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "about": wl.about, "n_q": d.n_q, "q_pos0": d.q_pos0,
+                   "ctx_len": d.ctx_len, "top_k": d.top_k, "n_heads": d.n_heads,
+                   "d_latent": d.d_latent, "d_rope": d.d_rope, "n_idx_heads": d.n_idx_heads,
+                   "d_idx": d.d_idx, "parallelism": f"dp{world} (independent chunks)",
+                   "l2": "flushed: 256 MB write between timed steps"},
+        "tflops": tflops,
+        "pct_of_measured_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "pct_of_spec_bf16_peak": 100.0 * tflops / SPEC_BF16_TFLOPS,
+        "useful_flop_per_step": fl["total"],
+        "per_kernel_ms": per_kernel,
+        "e2e": {"value": world * d.n_q / (e2e_ms / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": KERNELS_PER_LAYER * args.steps,
+        "roofline": roof,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(d, x, args.cpu_rows)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------- CPU reference
+
+
+def oracle_sample(d, x, n_rows):
+    """Times the float64 oracle on n_rows query rows spread over the chunk."""
+    import oracle
+
+    rows = np.linspace(0, d.n_q - 1, n_rows).round().astype(np.int32)
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.prefill_layer(d, **x, rows=rows, n_threads=cores)
+    dt = time.perf_counter() - t0
+    return n_rows / dt, cores, dt
+
+
+def cpu_baseline(d, x, n_rows):
+    qps, cores, dt = oracle_sample(d, x, n_rows)
+    return {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_rows} query rows spread over the chunk (float64 oracle, "
+                      f"{dt:.1f} s wall)"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    wl = workloads.BY_NAME[args.workload]
+    d = wl.dims
+    w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
+    x = workloads.generate(d, wl.seed, wl.kind, w_mode)
+    rows_per_step = args.cpu_rows
+    for _ in range(args.warmup):
+        oracle_sample(d, x, max(1, rows_per_step // 4))
+    times = []
+    cores = os.cpu_count() or 1
+    for _ in range(args.steps):
+        _, cores, dt = oracle_sample(d, x, rows_per_step)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = rows_per_step / (ms / 1e3)
+    result = {
+        "impl": "reference", "metric": "DSA prefill queries/s per layer", "value": value,
+        "unit": "queries/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "about": wl.about, "n_q": d.n_q, "ctx_len": d.ctx_len,
+                   "top_k": d.top_k},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows_per_step} query rows per step"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="chunk8k_ctx17k", choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--cpu-rows", type=int, default=48,
+                    help="query rows of the bounded CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/* dsa.h -- C ABI of the B200 (sm_100a) DSA sparse-attention prefill library.
+ *
+ * One call processes one prefill chunk of n_q queries against a cache that
+ * already holds the chunk's own rows. Query i sits at absolute position
+ * t = q_pos0 + i and sees cache rows s = 0..t.
+ *
+ * Where the operations come from. The feedman.me post feedman.me/posts/wy2HU
+ * (an M3 Ultra + M5 Ultra prefill/decode split for GLM-5.3-Flash) profiles the
+ * layer in its per-component prefill table (rows "DSA indexer" and "DSA
+ * sparse-attention core"), calls the attention step a per-query top-2048
+ * gather kernel (paragraph after the table), describes it as gathering each
+ * query's 2,048 keys for dot products (paragraph "Two levers fell out of
+ * this"), and gives the 512-wide latent KV ("Why the hand-off is cheap"). The
+ * pages print no formula; the definitions below are the plainest reading of
+ * DeepSeek-style sparse attention that agrees with them.
+ *
+ * Conventions shared by every entry point
+ *  - bf16 tensors are passed as uint16_t bit patterns; float tensors are IEEE
+ *    float32; every tensor is dense, row-major, in device memory, and its base
+ *    address is 16-byte aligned.
+ *  - The caller owns all memory, including the workspace. The library never
+ *    allocates or frees memory and never synchronizes the stream, except
+ *    dsa_device_status(), which exists to do exactly that.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    is the legacy default stream). The returned status covers argument
+ *    checks and kernel launch only. A device-side failure (a bounded wait that
+ *    gave up, or an index out of range) is recorded in the workspace's status
+ *    word and reported by dsa_device_status(). Every call clears that word
+ *    first, so it always describes the latest call that used the workspace.
+ *  - Calls that share a workspace must not overlap on the GPU (use one stream,
+ *    or one workspace per stream).
+ *  - Argument errors are returned before anything is launched; outputs are
+ *    then left untouched.
+ *  - n_q == 0 is valid and launches nothing.
+ *  - Inputs must be finite (no NaN or Inf).
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Shapes of one prefill chunk. */
+typedef struct dsa_dims {
+  int32_t n_q;         /* queries in the chunk, >= 0                                  */
+  int32_t q_pos0;      /* absolute position of query 0, >= 0                          */
+  int32_t ctx_len;     /* cache rows T, q_pos0 + n_q <= T <= DSA_MAX_CTX              */
+  int32_t n_heads;     /* attention heads H                                           */
+  int32_t d_latent;    /* latent width Dc (the attention value is the latent row)     */
+  int32_t d_rope;      /* rotary width Dr (keys only; already rotated)                */
+  int32_t n_idx_heads; /* indexer heads H_I (query side; one shared key per row)      */
+  int32_t d_idx;       /* indexer head width D_I                                      */
+  int32_t top_k;       /* keys kept per query, 1..DSA_MAX_TOPK                        */
+  float softmax_scale; /* multiplies the attention logits                             */
+  uint32_t flags;      /* must be 0                                                   */
+} dsa_dims;
+
+/* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):
+ *   (n_heads, d_latent, d_rope)  in {(4, 64, 16), (32, 512, 64)}
+ *   (n_idx_heads, d_idx)         in {(2, 32), (32, 128)}
+ *   1 <= top_k <= 2048, ctx_len <= 49152                                       */
+#define DSA_MAX_TOPK 2048
+#define DSA_MAX_CTX 49152
+
+typedef int32_t dsa_status;
+#define DSA_OK 0
+#define DSA_ERR_NULL (-1)      /* a required pointer is NULL                          */
+#define DSA_ERR_ALIGN (-2)     /* a pointer is not 16-byte aligned, or ld % 4 != 0    */
+#define DSA_ERR_DIMS (-3)      /* unsupported or inconsistent shape, or flags != 0     */
+#define DSA_ERR_CAUSAL (-4)    /* q_pos0 + n_q > ctx_len                               */
+#define DSA_ERR_WORKSPACE (-5) /* workspace NULL or smaller than dsa_workspace_size()  */
+#define DSA_ERR_TIMEOUT (-6)   /* a device-side bounded wait gave up                   */
+#define DSA_ERR_CUDA (-7)      /* CUDA runtime or launch error                         */
+#define DSA_ERR_DEVICE (-8)    /* current device is not sm_100 (B200)                  */
+#define DSA_ERR_RANGE (-9)     /* device found a selected index outside 0..t           */
+
+/* Which call a workspace is for. */
+#define DSA_WS_INDEX_SCORES 0
+#define DSA_WS_TOPK 1
+#define DSA_WS_ATTN 2
+#define DSA_WS_LAYER 3
+
+/* Bytes of device workspace the call `which` needs for these dims (0 on bad
+ * arguments). The first 256 bytes of every workspace hold the device status
+ * word and per-call scalars; dsa_prefill_layer adds the float32 score matrix
+ * [n_q, round_up(ctx_len, 128)] and an int32 selection [n_q, top_k] after
+ * them. Workspace contents need no initialisation and are not preserved
+ * between calls. */
+size_t dsa_workspace_size(const dsa_dims* dims, int32_t which);
+
+/* Lightning-indexer scores (component-table row "DSA indexer" of the feedman.me
+ * post). For query row i at position t and cache row s <= t:
+ *     I[i,s] = sum_j w_idx[i,j] * ReLU( sum_c q_idx[i,j,c] * k_idx[s,c] )
+ * computed with bf16 products, float32 accumulation on tensor cores and a
+ * float32 head sum.
+ *   q_idx   bf16  [n_q, n_idx_heads, d_idx]
+ *   k_idx   bf16  [ctx_len, d_idx]        one key per cache row, shared by heads
+ *   w_idx   f32   [n_q, n_idx_heads]
+ *   scores  f32   [n_q, ld_scores], ld_scores >= ctx_len, ld_scores % 4 == 0.
+ *           Row i holds I[i,s] for s <= t; entries s > t are not written.
+ * Errors: DSA_ERR_NULL, _ALIGN, _DIMS, _CAUSAL, _WORKSPACE, _DEVICE, _CUDA. */
+dsa_status dsa_index_scores(const dsa_dims* dims, const uint16_t* q_idx, const uint16_t* k_idx,
+                            const float* w_idx, float* scores, int64_t ld_scores,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Per-query top-k selection (the "per-query top-2048" step of the feedman.me
+ * post, paragraph after the component table). Among s = 0..t, keys are
+ * ordered by score descending and then index ascending; the first
+ * min(top_k, t+1) are kept and written in ascending index order, the unused
+ * tail of the row holding -1.
+ *   scores  f32   [n_q, ld_scores] as written by dsa_index_scores (only
+ *                 entries s <= t are read)
+ *   idx     int32 [n_q, top_k] (output)
+ * With q_idx, k_idx and w_idx all NULL the order is that of the given float32
+ * scores. With all three given, the order is that of the float64 definition
+ *     d_j = sum_c q*k (float64, in c order), r_j = max(d_j, +0),
+ *     score = sum_j w_j * r_j (float64, in j order, no fused multiply-add)
+ * which the kernel reproduces exactly: float32 scores within a proven error
+ * bound decide every key except those whose bound straddles the k-th score,
+ * and those are re-scored in float64 in that order. Giving only some of the
+ * three is DSA_ERR_NULL.
+ * Errors: DSA_ERR_NULL, _ALIGN, _DIMS, _CAUSAL, _WORKSPACE, _DEVICE, _CUDA. */
+dsa_status dsa_topk_select(const dsa_dims* dims, const float* scores, int64_t ld_scores,
+                           const uint16_t* q_idx, const uint16_t* k_idx, const float* w_idx,
+                           int32_t* idx, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Sparse MLA-style attention over the selected keys (component-table row "DSA
+ * sparse-attention core" of the feedman.me post). For query row i, head h and
+ * the keys S listed in idx[i,:] (entries < 0 are skipped):
+ *     z_s = softmax_scale * ( q[i,h,:Dc] . latent[s,:] + q[i,h,Dc:] . rope[s,:] )
+ *     out[i,h,:] = sum_{s in S} softmax(z)_s * latent[s,:]
+ *     lse[i,h]   = log sum_{s in S} exp(z_s)
+ * bf16 operands, float32 accumulation, bf16 output rounded to nearest even.
+ * A row with no valid key gets out = 0 and lse = -inf.
+ *   q      bf16  [n_q, n_heads, d_latent + d_rope]
+ *   latent bf16  [ctx_len, d_latent]
+ *   rope   bf16  [ctx_len, d_rope]
+ *   idx    int32 [n_q, top_k], every valid entry in 0..ctx_len-1
+ *   out    bf16  [n_q, n_heads, d_latent] (output)
+ *   lse    f32   [n_q, n_heads] (output) or NULL
+ * Out-of-range indices are not read; they set DSA_ERR_RANGE in the workspace
+ * status and that key is skipped.
+ * Errors: DSA_ERR_NULL, _ALIGN, _DIMS, _CAUSAL, _WORKSPACE, _DEVICE, _CUDA. */
+dsa_status dsa_sparse_attn_prefill(const dsa_dims* dims, const uint16_t* q,
+                                   const uint16_t* latent, const uint16_t* rope,
+                                   const int32_t* idx, uint16_t* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* The whole layer on one stream: indexer scores -> exact top-k (float64
+ * order, as in dsa_topk_select with the indexer inputs given) -> sparse
+ * attention. idx_out ([n_q, top_k]) and lse may be NULL. The float32 score
+ * matrix lives in the workspace. */
+dsa_status dsa_prefill_layer(const dsa_dims* dims, const uint16_t* q, const uint16_t* latent,
+                             const uint16_t* rope, const uint16_t* q_idx,
+                             const uint16_t* k_idx, const float* w_idx, uint16_t* out,
+                             float* lse, int32_t* idx_out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* Synchronizes `stream`, returns the device status word of `workspace`
+ * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_RANGE) and clears it. */
+dsa_status dsa_device_status(void* workspace, void* stream);
+
+/* Static text for a status code. */
+const char* dsa_status_string(dsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,225 @@
+// dsa_api.cu -- the C ABI: argument checks, workspace layout and launch order.
+//
+// Every entry point validates its arguments completely before it launches
+// anything (a lesson the TensorFold issue #743 thread draws from a sparse
+// attention kernel that launched past a hardware limit on some GPUs: here a
+// shape the kernels were not built for is an error, never a launch).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "dsa.h"
+#include "dsa_internal.cuh"
+
+using dsa::WsHeader;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_device_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+
+dsa_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_DEVICE;
+  if (g_device_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    g_device_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_device_ok[dev] == 1 ? DSA_OK : DSA_ERR_DEVICE;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool attn_shape_ok(const dsa_dims& d) {
+  return (d.n_heads == 4 && d.d_latent == 64 && d.d_rope == 16) ||
+         (d.n_heads == 32 && d.d_latent == 512 && d.d_rope == 64);
+}
+
+bool indexer_shape_ok(const dsa_dims& d) {
+  return (d.n_idx_heads == 2 && d.d_idx == 32) || (d.n_idx_heads == 32 && d.d_idx == 128);
+}
+
+// Common shape checks. `need_attn` / `need_indexer` select which head shapes
+// the call uses.
+dsa_status check_dims(const dsa_dims* d, bool need_attn, bool need_indexer) {
+  if (!d) return DSA_ERR_NULL;
+  if (d->flags != 0u) return DSA_ERR_DIMS;
+  if (d->n_q < 0 || d->q_pos0 < 0 || d->ctx_len < 1 || d->ctx_len > DSA_MAX_CTX)
+    return DSA_ERR_DIMS;
+  if (d->top_k < 1 || d->top_k > DSA_MAX_TOPK) return DSA_ERR_DIMS;
+  if (need_attn && !attn_shape_ok(*d)) return DSA_ERR_DIMS;
+  if (need_indexer && !indexer_shape_ok(*d)) return DSA_ERR_DIMS;
+  if (need_attn && !(d->softmax_scale > 0.0f && d->softmax_scale < 1e30f)) return DSA_ERR_DIMS;
+  if (static_cast<int64_t>(d->q_pos0) + d->n_q > d->ctx_len) return DSA_ERR_CAUSAL;
+  return DSA_OK;
+}
+
+int64_t layer_ld(const dsa_dims& d) { return (static_cast<int64_t>(d.ctx_len) + 127) / 128 * 128; }
+
+size_t layer_scores_bytes(const dsa_dims& d) {
+  return static_cast<size_t>(d.n_q) * layer_ld(d) * sizeof(float);
+}
+
+int32_t* layer_idx_region(void* ws, const dsa_dims& d) {
+  return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes +
+                                    layer_scores_bytes(d));
+}
+
+dsa_status check_ws(const dsa_dims& d, int which, void* ws, size_t bytes) {
+  if (!ws) return DSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return DSA_ERR_ALIGN;
+  if (bytes < dsa_workspace_size(&d, which)) return DSA_ERR_WORKSPACE;
+  return DSA_OK;
+}
+
+dsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+dsa_status clear_header(void* ws, cudaStream_t st) {
+  return from_cuda(cudaMemsetAsync(ws, 0, dsa::kWsHeaderBytes, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_workspace_size(const dsa_dims* d, int32_t which) {
+  if (!d || d->n_q < 0 || d->ctx_len < 1) return 0;
+  switch (which) {
+    case DSA_WS_INDEX_SCORES:
+    case DSA_WS_TOPK:
+    case DSA_WS_ATTN:
+      return dsa::kWsHeaderBytes;
+    case DSA_WS_LAYER:
+      return dsa::kWsHeaderBytes + layer_scores_bytes(*d) +
+             static_cast<size_t>(d->n_q) * d->top_k * sizeof(int32_t);
+    default:
+      return 0;
+  }
+}
+
+dsa_status dsa_index_scores(const dsa_dims* d, const uint16_t* q_idx, const uint16_t* k_idx,
+                            const float* w_idx, float* scores, int64_t ld, void* ws,
+                            size_t ws_bytes, void* stream) {
+  dsa_status s = check_dims(d, false, true);
+  if (s != DSA_OK) return s;
+  if (!q_idx || !k_idx || !w_idx || !scores) return DSA_ERR_NULL;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(scores) ||
+      ld % 4 != 0)
+    return DSA_ERR_ALIGN;
+  if (ld < d->ctx_len) return DSA_ERR_DIMS;
+  if ((s = check_ws(*d, DSA_WS_INDEX_SCORES, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  return from_cuda(dsa::launch_index_scores(*d, q_idx, k_idx, w_idx, scores, ld,
+                                            static_cast<WsHeader*>(ws), st));
+}
+
+dsa_status dsa_topk_select(const dsa_dims* d, const float* scores, int64_t ld,
+                           const uint16_t* q_idx, const uint16_t* k_idx, const float* w_idx,
+                           int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  const int given = (q_idx != nullptr) + (k_idx != nullptr) + (w_idx != nullptr);
+  dsa_status s = check_dims(d, false, given == 3);
+  if (s != DSA_OK) return s;
+  if (!scores || !idx || (given != 0 && given != 3)) return DSA_ERR_NULL;
+  if (!aligned16(scores) || !aligned16(idx) || ld % 4 != 0) return DSA_ERR_ALIGN;
+  if (given == 3 && (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w_idx)))
+    return DSA_ERR_ALIGN;
+  if (ld < d->ctx_len) return DSA_ERR_DIMS;
+  if ((s = check_ws(*d, DSA_WS_TOPK, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  if (given == 3) {
+    cudaError_t e = dsa::launch_key_norm_max(*d, k_idx, h, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return from_cuda(dsa::launch_topk(*d, scores, ld, q_idx, k_idx, w_idx, idx, h, st));
+}
+
+dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
+                                   const uint16_t* rope, const int32_t* idx, uint16_t* out,
+                                   float* lse, void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_dims(d, true, false);
+  if (s != DSA_OK) return s;
+  if (!q || !latent || !rope || !idx || !out) return DSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(idx) ||
+      !aligned16(out) || (lse && !aligned16(lse)))
+    return DSA_ERR_ALIGN;
+  if ((s = check_ws(*d, DSA_WS_ATTN, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse,
+                                           static_cast<WsHeader*>(ws), st));
+}
+
+dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
+                             const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
+                             const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
+                             void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_dims(d, true, true);
+  if (s != DSA_OK) return s;
+  if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
+      !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(out) || (lse && !aligned16(lse)) ||
+      (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGN;
+  if ((s = check_ws(*d, DSA_WS_LAYER, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes);
+  const int64_t ld = layer_ld(*d);
+  // The selection goes to the caller's idx_out when given, else to the
+  // workspace region after the score matrix.
+  int32_t* idx = idx_out ? idx_out : layer_idx_region(ws, *d);
+  cudaError_t e = dsa::launch_index_scores(*d, q_idx, k_idx, w_idx, scores, ld, h, st);
+  if (e == cudaSuccess) e = dsa::launch_key_norm_max(*d, k_idx, h, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  e = dsa::launch_topk(*d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, h, st));
+}
+
+dsa_status dsa_device_status(void* ws, void* stream) {
+  if (!ws) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  unsigned int code = 0;
+  if (cudaMemcpy(&code, ws, sizeof code, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (code != 0 && cudaMemset(ws, 0, 2 * sizeof(unsigned int)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (code == dsa::kDevTimeout) return DSA_ERR_TIMEOUT;
+  if (code == dsa::kDevRange) return DSA_ERR_RANGE;
+  return code == 0 ? DSA_OK : DSA_ERR_CUDA;
+}
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_NULL: return "a required pointer is NULL";
+    case DSA_ERR_ALIGN: return "a pointer is not 16-byte aligned, or ld is not a multiple of 4";
+    case DSA_ERR_DIMS: return "unsupported or inconsistent shape, or nonzero flags";
+    case DSA_ERR_CAUSAL: return "q_pos0 + n_q exceeds ctx_len";
+    case DSA_ERR_WORKSPACE: return "workspace missing or smaller than dsa_workspace_size()";
+    case DSA_ERR_TIMEOUT: return "a device-side bounded wait gave up";
+    case DSA_ERR_CUDA: return "CUDA runtime or launch error";
+    case DSA_ERR_DEVICE: return "current device is not an sm_100 (B200) GPU";
+    case DSA_ERR_RANGE: return "a selected index was outside the causal range";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

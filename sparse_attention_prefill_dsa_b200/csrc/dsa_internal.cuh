@@ -1,0 +1,59 @@
+// dsa_internal.cuh -- shared definitions of the CUDA library (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dsa.h"
+
+namespace dsa {
+
+// First 256 bytes of every workspace.
+struct WsHeader {
+  unsigned int status;        // 0 or a positive code: kDevTimeout / kDevRange
+  unsigned int status_info;   // first failing site (kernel-specific)
+  unsigned long long kmax_bits;  // float64 bit pattern of max_s ||k_idx[s]||_2 (>= 0)
+  unsigned char pad[240];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+constexpr unsigned int kDevTimeout = 1;
+constexpr unsigned int kDevRange = 2;
+constexpr unsigned int kDevInternal = 3;  // an internal consistency check failed
+constexpr size_t kWsHeaderBytes = 256;
+
+// Records the first device-side failure in the workspace header.
+__device__ __forceinline__ void report(WsHeader* ws, unsigned int code, unsigned int info) {
+  if (atomicCAS(&ws->status, 0u, code) == 0u) ws->status_info = info;
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) {
+  return __uint_as_float(static_cast<unsigned int>(h) << 16);
+}
+
+__device__ __forceinline__ double bf16_to_f64(uint16_t h) {
+  return static_cast<double>(__uint_as_float(static_cast<unsigned int>(h) << 16));
+}
+
+// float32 -> bf16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  unsigned int b = __float_as_uint(f);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return static_cast<uint16_t>(b >> 16);
+}
+
+// Launchers (one per kernel family), defined in the .cu files. Each returns
+// cudaGetLastError() after its launches.
+cudaError_t launch_index_scores(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_idx,
+                                const float* w_idx, float* scores, int64_t ld, WsHeader* ws,
+                                cudaStream_t st);
+cudaError_t launch_key_norm_max(const dsa_dims& d, const uint16_t* k_idx, WsHeader* ws,
+                                cudaStream_t st);
+cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld,
+                        const uint16_t* q_idx, const uint16_t* k_idx, const float* w_idx,
+                        int32_t* idx, WsHeader* ws, cudaStream_t st);
+cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
+                               const uint16_t* rope, const int32_t* idx, uint16_t* out,
+                               float* lse, WsHeader* ws, cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,123 @@
+"""The C ABI on the CPU: the library loads, exports every function include/dsa.h
+declares, sizes workspaces, and rejects bad arguments before touching a device.
+No test here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import workloads
+from workloads import make_dims
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    from sparse_attention_prefill_dsa_b200 import build
+
+    build.build()
+    import sparse_attention_prefill_dsa_b200 as m
+
+    m.library()
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
+              "dsa_prefill_layer", "dsa_workspace_size", "dsa_status_string",
+              "dsa_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(dsa):
+    lib = ctypes.CDLL(dsa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in dsa.EXPORTED or name.startswith("dsa_"), name
+
+
+def test_binding_has_a_function_per_symbol(dsa):
+    for name in declared_functions():
+        assert callable(getattr(dsa, name)), name
+
+
+def test_dims_struct_layout_matches_header(dsa):
+    assert ctypes.sizeof(dsa.dsa_dims) == 11 * 4
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct dsa_dims"):text.index("} dsa_dims;")]
+    fields = re.findall(r"\b(?:int32_t|uint32_t|float)\s+([a-z_0-9]+);", body)
+    assert fields == [f for f, _ in dsa.dsa_dims._fields_]
+
+
+def test_status_codes_and_strings(dsa):
+    text = open(HEADER).read()
+    for name, val in re.findall(r"#define (DSA_(?:OK|ERR_[A-Z]+))\s+\(?(-?\d+)\)?", text):
+        assert getattr(dsa, name) == int(val), name
+        assert dsa.dsa_status_string(int(val))
+    assert dsa.dsa_status_string(12345) == "unknown status"
+
+
+def test_workspace_sizes(dsa):
+    d = workloads.BY_NAME["chunk8k_ctx17k"].dims
+    assert dsa.dsa_workspace_size(d, dsa.DSA_WS_TOPK) == 256
+    ld = (d.ctx_len + 127) // 128 * 128
+    assert dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER) == 256 + d.n_q * ld * 4 + d.n_q * d.top_k * 4
+    assert dsa.dsa_workspace_size(d, 99) == 0
+
+
+FAKE = 1 << 20  # an aligned, never dereferenced address
+
+
+def _layer(dsa, d, **over):
+    a = dict(q=FAKE, latent=FAKE, rope=FAKE, q_idx=FAKE, k_idx=FAKE, w_idx=FAKE, out=FAKE,
+             lse=None, idx_out=None, workspace=FAKE)
+    a.update(over)
+    nbytes = over.pop("workspace_bytes", dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER))
+    return dsa.dsa_prefill_layer(d, a["q"], a["latent"], a["rope"], a["q_idx"], a["k_idx"],
+                                 a["w_idx"], a["out"], a["lse"], a["idx_out"], a["workspace"],
+                                 workspace_bytes=nbytes, stream=0)
+
+
+def test_host_validation_before_any_device_call(dsa):
+    d = workloads.BY_NAME["chunk2k_ctx8k"].dims
+    assert _layer(dsa, d, q=None) == dsa.DSA_ERR_NULL
+    assert _layer(dsa, d, latent=FAKE + 8) == dsa.DSA_ERR_ALIGN
+    assert _layer(dsa, d, workspace=None) == dsa.DSA_ERR_WORKSPACE
+    assert _layer(dsa, d, workspace_bytes=100) == dsa.DSA_ERR_WORKSPACE
+    bad = dsa.make_dims(d)
+    bad.n_q = d.n_q + 1
+    assert _layer(dsa, bad) == dsa.DSA_ERR_CAUSAL
+    for field, val in (("top_k", 0), ("top_k", 2049), ("ctx_len", 49153), ("n_heads", 8),
+                       ("d_latent", 256), ("n_idx_heads", 64), ("flags", 2), ("n_q", -1),
+                       ("softmax_scale", 0.0)):
+        bad = dsa.make_dims(d)
+        setattr(bad, field, val)
+        assert _layer(dsa, bad) in (dsa.DSA_ERR_DIMS, dsa.DSA_ERR_CAUSAL), field
+    # top-k: indexer inputs all or none
+    ws = dsa.dsa_workspace_size(d, dsa.DSA_WS_TOPK)
+    assert dsa.dsa_topk_select(d, FAKE, d.ctx_len, FAKE, None, None, FAKE, FAKE, ws, 0) == \
+        dsa.DSA_ERR_NULL
+    assert dsa.dsa_topk_select(d, FAKE, d.ctx_len + 2, None, None, None, FAKE, FAKE, ws, 0) == \
+        dsa.DSA_ERR_ALIGN
+    assert dsa.dsa_index_scores(d, FAKE, FAKE, FAKE, FAKE, d.ctx_len - 4, FAKE, ws, 0) == \
+        dsa.DSA_ERR_DIMS
+
+
+def test_valid_call_without_gpu_reports_device_error(dsa):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    d = make_dims(4, 0, 4, 4, 64, 16, 2, 32, 2)
+    st = _layer(dsa, d)
+    assert st in (dsa.DSA_ERR_CUDA, dsa.DSA_ERR_DEVICE)

@@ -1,0 +1,276 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Bar: selected index sets bit-exact; attention outputs within max-abs 2e-2 and
+relative L2 5e-3 of the oracle (bf16 in/out, float32 accumulation).
+Full element-wise comparisons run on reduced chunks of each workload (the
+oracle finishes them in seconds; they still span several tiles and end on a
+ragged tail); the full-size workloads, in the launch configuration the bench
+times, are compared on sampled query rows that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+
+import workloads
+from workloads import make_dims
+
+from dsa_test_util import (assert_attn_close, attn_errors, dev, dev_bf16, empty_bf16,
+                           host_bf16_as_f32, run_layer, stage, workspace)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_attention_prefill_dsa_b200 as m
+
+    m.library()
+    return m
+
+
+def _reduced(name, n_q, w_mode=None):
+    wl = workloads.BY_NAME[name]
+    d0 = wl.dims
+    d = make_dims(n_q, d0.ctx_len - n_q, d0.ctx_len, d0.n_heads, d0.d_latent, d0.d_rope,
+                  d0.n_idx_heads, d0.d_idx, d0.top_k, d0.softmax_scale)
+    if w_mode is None:
+        w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
+    return d, workloads.generate(d, wl.seed + 100, wl.kind, w_mode)
+
+
+def _compare_layer(oracle_lib, d, x, out, lse, idx, rows=None):
+    ref_out, ref_lse, ref_idx = oracle_lib.prefill_layer(d, **x, rows=rows)
+    sel = slice(None) if rows is None else rows
+    bad = np.nonzero(~np.all(idx[sel] == ref_idx, axis=1))[0]
+    assert bad.size == 0, f"{bad.size} rows differ in their selected sets, first row {bad[:4]}"
+    assert_attn_close(out[sel], ref_out)
+    finite = np.isfinite(ref_lse)
+    np.testing.assert_allclose(lse[sel][finite], ref_lse[finite], rtol=0, atol=2e-3)
+
+
+def test_layer_tiny_workload_full(dsa, oracle_lib):
+    d, x = workloads.workload_inputs("tiny_256q")
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    _compare_layer(oracle_lib, d, x, out, lse, idx)
+
+
+@pytest.mark.parametrize("name,n_q,w_mode", [
+    ("chunk2k_ctx8k", 157, None),
+    ("chunk8k_ctx17k", 131, None),
+    ("chunk16k_ctx48k", 40, None),
+    ("ties_4k_ctx8k", 149, None),
+    ("ties_4k_ctx8k", 77, "uniform"),
+])
+def test_layer_reduced_elementwise(dsa, oracle_lib, name, n_q, w_mode):
+    d, x = _reduced(name, n_q, w_mode)
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    _compare_layer(oracle_lib, d, x, out, lse, idx)
+
+
+@pytest.mark.parametrize("name,n_rows", [
+    ("chunk2k_ctx8k", 24), ("chunk8k_ctx17k", 24), ("chunk16k_ctx48k", 12), ("ties_4k_ctx8k", 24)])
+def test_layer_full_size_sampled_rows(dsa, oracle_lib, name, n_rows):
+    d, x = workloads.workload_inputs(name)
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    rng = np.random.default_rng(1234)
+    rows = np.unique(np.concatenate([[0, d.n_q - 1], rng.integers(0, d.n_q, n_rows - 2)]))
+    _compare_layer(oracle_lib, d, x, out, lse, idx, rows=rows.astype(np.int32))
+    # every row: a valid causal, ascending set of exactly min(k, t+1) keys
+    t = d.q_pos0 + np.arange(d.n_q)
+    assert np.all(np.diff(idx, axis=1) > 0)
+    assert np.all(idx[:, 0] >= 0) and np.all(idx.max(axis=1) <= t)
+
+
+def test_index_scores_within_certified_bound(dsa, oracle_lib):
+    """float32 indexer scores stay far inside the bound the exact top-k relies on."""
+    import torch
+
+    d, x = _reduced("chunk2k_ctx8k", 64)
+    xd = stage(x)
+    ld = (d.ctx_len + 3) // 4 * 4
+    sc = torch.full((d.n_q, ld), float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_INDEX_SCORES))
+    dsa.check(dsa.dsa_index_scores(d, xd["q_idx"], xd["k_idx"], xd["w_idx"], sc, ld, ws))
+    torch.cuda.synchronize()
+    f32 = sc.cpu().numpy()
+    ref = oracle_lib.index_scores(d, x["q_idx"], x["k_idx"], x["w_idx"])
+    qi = workloads.bf16_bits_to_f32(x["q_idx"]).astype(np.float64)
+    ki = workloads.bf16_bits_to_f32(x["k_idx"]).astype(np.float64)
+    A = (np.abs(x["w_idx"].astype(np.float64)) * np.linalg.norm(qi, axis=2)).sum(axis=1)
+    kmax = np.linalg.norm(ki, axis=1).max()
+    worst = 0.0
+    for i in range(d.n_q):
+        t = d.q_pos0 + i
+        err = np.abs(f32[i, : t + 1].astype(np.float64) - ref[i, : t + 1]).max()
+        worst = max(worst, err / (A[i] * kmax))
+    bound = 2.0 ** -14 + 2.0 ** -17
+    print(f"worst |F-X| / (A_t Kmax) = {worst:.3e} (bound {bound:.3e})")
+    assert worst <= bound / 16
+
+
+def test_topk_on_float32_scores_is_bitexact(dsa, oracle_lib):
+    """With no indexer inputs the select orders the given float32 scores."""
+    import torch
+
+    rng = np.random.default_rng(7)
+    d = make_dims(300, 700, 1000, 32, 512, 64, 32, 128, 256)
+    ld = 1000
+    s32 = rng.integers(0, 50, size=(d.n_q, ld)).astype(np.float32) * np.float32(0.125)
+    s32[:, ::7] = -s32[:, ::7]           # negatives too
+    s32[5, :] = 0.0                      # a row of exact ties
+    s32[6, ::2] = -0.0                   # -0 and +0 tie
+    idx = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_TOPK))
+    dsa.check(dsa.dsa_topk_select(d, dev(s32), ld, None, None, None, idx, ws))
+    dsa.check(dsa.dsa_device_status(ws))
+    ref = oracle_lib.topk_select(d, s32)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_exact_mode_on_gpu_scores(dsa, oracle_lib):
+    """dsa_topk_select with indexer inputs reproduces the float64 order."""
+    import torch
+
+    d, x = _reduced("ties_4k_ctx8k", 96)
+    xd = stage(x)
+    ld = d.ctx_len
+    sc = torch.empty(d.n_q, ld, dtype=torch.float32, device="cuda")
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_TOPK))
+    dsa.check(dsa.dsa_index_scores(d, xd["q_idx"], xd["k_idx"], xd["w_idx"], sc, ld, ws))
+    idx = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
+    dsa.check(dsa.dsa_topk_select(d, sc, ld, xd["q_idx"], xd["k_idx"], xd["w_idx"], idx, ws))
+    dsa.check(dsa.dsa_device_status(ws))
+    ref = oracle_lib.topk_select(d, oracle_lib.index_scores(d, x["q_idx"], x["k_idx"], x["w_idx"]))
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
+def test_sparse_attn_entry_point_on_given_sets(dsa, oracle_lib):
+    """dsa_sparse_attn_prefill on oracle-chosen sets, with padding and shuffled order."""
+    import torch
+
+    d, x = _reduced("chunk2k_ctx8k", 50)
+    _, _, ref_idx = oracle_lib.prefill_layer(d, **x)
+    rng = np.random.default_rng(3)
+    idx = np.stack([rng.permutation(r) for r in ref_idx]).astype(np.int32)
+    idx[7, 100:] = -1                     # a row with a short list
+    idx[8, :] = -1                        # a row with no key: out 0, lse -inf
+    ref_out, ref_lse = oracle_lib.sparse_attn(d, x["q"], x["latent"], x["rope"], idx)
+    xd = stage(x)
+    out = empty_bf16(d.n_q, d.n_heads, d.d_latent)
+    lse = torch.empty(d.n_q, d.n_heads, dtype=torch.float32, device="cuda")
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_ATTN))
+    dsa.check(dsa.dsa_sparse_attn_prefill(d, xd["q"], xd["latent"], xd["rope"], dev(idx), out,
+                                          lse, ws))
+    dsa.check(dsa.dsa_device_status(ws))
+    o = host_bf16_as_f32(out)
+    assert_attn_close(o, ref_out)
+    assert np.all(o[8] == 0) and np.all(np.isneginf(lse.cpu().numpy()[8]))
+
+
+# ----------------------------------------------------------------- edge cases
+
+
+def test_empty_chunk_launches_nothing(dsa):
+    import torch
+
+    d = make_dims(0, 10, 10, 32, 512, 64, 32, 128, 2048)
+    one = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(16, dtype=torch.float32, device="cuda")
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER))
+    assert dsa.dsa_prefill_layer(d, one, one, one, one, one, w, one, None, None, ws) == dsa.DSA_OK
+    assert dsa.dsa_device_status(ws) == dsa.DSA_OK
+
+
+@pytest.mark.parametrize("n_q,q_pos0,T,k", [
+    (1, 0, 1, 2048),        # one query that sees only itself
+    (3, 0, 3, 1),           # k = 1
+    (70, 930, 1000, 500),   # ragged context, partial key tiles
+    (33, 0, 33, 2048),      # every row keeps all causal keys, -1 padding
+])
+def test_layer_edge_shapes(dsa, oracle_lib, n_q, q_pos0, T, k):
+    d = make_dims(n_q, q_pos0, T, 32, 512, 64, 32, 128, k)
+    x = workloads.generate(d, 21, "normal", "uniform")
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    _compare_layer(oracle_lib, d, x, out, lse, idx)
+
+
+def test_layer_all_keys_tied(dsa, oracle_lib):
+    """Identical indexer keys: every score of a row ties, so the band holds
+    the whole row (larger than the kernel's band cache) and the lowest
+    indices must win."""
+    d = make_dims(6, 6000, 6006, 32, 512, 64, 32, 128, 2048)
+    x = workloads.generate(d, 22, "normal", "uniform")
+    x["k_idx"] = np.ascontiguousarray(np.broadcast_to(x["k_idx"][:1], x["k_idx"].shape))
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    for i in range(d.n_q):
+        assert idx[i].tolist() == list(range(d.top_k))
+    _compare_layer(oracle_lib, d, x, out, lse, idx)
+
+
+def test_layer_zero_weights(dsa, oracle_lib):
+    d = make_dims(20, 980, 1000, 32, 512, 64, 32, 128, 300)
+    x = workloads.generate(d, 23, "normal", "uniform")
+    x["w_idx"] = np.zeros_like(x["w_idx"])
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    assert np.all(idx == np.arange(d.top_k)[None, :])
+    _compare_layer(oracle_lib, d, x, out, lse, idx)
+
+
+def test_chunk_split_is_invariant(dsa):
+    """Two half chunks give the same selections and bit-identical outputs."""
+    d, x = _reduced("chunk2k_ctx8k", 128)
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    h = d.n_q // 2
+    for part in range(2):
+        sl = slice(part * h, (part + 1) * h)
+        dp = make_dims(h, d.q_pos0 + part * h, d.ctx_len, d.n_heads, d.d_latent, d.d_rope,
+                       d.n_idx_heads, d.d_idx, d.top_k, d.softmax_scale)
+        xp = dict(x)
+        for key in ("q", "q_idx", "w_idx"):
+            xp[key] = np.ascontiguousarray(x[key][sl])
+        o, l, ix = run_layer(dsa, dp, stage(xp))
+        assert np.array_equal(ix, idx[sl])
+        assert np.array_equal(o, out[sl])
+        assert np.array_equal(l, lse[sl])
+
+
+def test_out_of_range_index_is_reported(dsa):
+    import torch
+
+    d, x = _reduced("chunk2k_ctx8k", 4)
+    xd = stage(x)
+    idx = np.tile(np.arange(d.top_k, dtype=np.int32), (d.n_q, 1))
+    idx[2, 5] = d.ctx_len + 7
+    out = empty_bf16(d.n_q, d.n_heads, d.d_latent)
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_ATTN))
+    dsa.check(dsa.dsa_sparse_attn_prefill(d, xd["q"], xd["latent"], xd["rope"], dev(idx), out,
+                                          None, ws))
+    assert dsa.dsa_device_status(ws) == dsa.DSA_ERR_RANGE
+    assert dsa.dsa_device_status(ws) == dsa.DSA_OK  # cleared by the read
+
+
+def test_argument_errors_launch_nothing(dsa):
+    import torch
+
+    d, x = _reduced("chunk2k_ctx8k", 8)
+    xd = stage(x)
+    out = torch.full((d.n_q, d.n_heads, d.d_latent), 3.0, dtype=torch.bfloat16, device="cuda")
+    nbytes = dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER)
+    ws = workspace(nbytes)
+    args = [xd["q"], xd["latent"], xd["rope"], xd["q_idx"], xd["k_idx"], xd["w_idx"], out, None,
+            None, ws]
+    assert dsa.dsa_prefill_layer(d, *args[:6], None, None, None, ws) == dsa.DSA_ERR_NULL
+    bad = list(args); bad[0] = xd["q"].data_ptr() + 2
+    assert dsa.dsa_prefill_layer(d, *bad) == dsa.DSA_ERR_ALIGN
+    assert dsa.dsa_prefill_layer(d, *args, workspace_bytes=nbytes - 1) == dsa.DSA_ERR_WORKSPACE
+    for field, val, code in (("top_k", 4096, dsa.DSA_ERR_DIMS), ("n_heads", 16, dsa.DSA_ERR_DIMS),
+                             ("d_idx", 64, dsa.DSA_ERR_DIMS), ("flags", 1, dsa.DSA_ERR_DIMS),
+                             ("n_q", d.n_q + 1, dsa.DSA_ERR_CAUSAL)):
+        dd = dsa.make_dims(d)
+        setattr(dd, field, val)
+        assert dsa.dsa_prefill_layer(dd, *args) == code
+    torch.cuda.synchronize()
+    assert torch.all(out == 3.0)  # nothing ran
