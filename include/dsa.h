@@ -77,6 +77,8 @@ typedef int32_t dsa_status;
 #define DSA_ERR_CUDA (-7)      /* CUDA runtime or launch error                         */
 #define DSA_ERR_DEVICE (-8)    /* current device is not sm_100 (B200)                  */
 #define DSA_ERR_RANGE (-9)     /* device found a selected index outside 0..t           */
+#define DSA_ERR_SCRATCH_LIMIT (-10) /* dsa_prefill_layer_noalloc: the chunk needs more
+                                       scratch than DSA_NOALLOC_SCRATCH_BYTES             */
 
 /* Which call a workspace is for. */
 #define DSA_WS_INDEX_SCORES 0
@@ -160,6 +162,35 @@ dsa_status dsa_prefill_layer(const dsa_dims* dims, const uint16_t* q, const uint
                              const uint16_t* k_idx, const float* w_idx, uint16_t* out,
                              float* lse, int32_t* idx_out, void* workspace,
                              size_t workspace_bytes, void* stream);
+
+/* The whole layer, as dsa_prefill_layer, for callers that cannot allocate
+ * device memory: code that runs inside another engine's plugin or callback and
+ * is handed only its input and output buffers, or code that must not touch the
+ * device allocator while a memory pool is shared or being captured. The pages
+ * have no counterpart to this call; it exists for such callers only.
+ *
+ * The scratch (score rows, selections, status word) lives in a static device
+ * array of DSA_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads the
+ * library holds until the process exits. The call allocates nothing:
+ *  - chunks whose dsa_workspace_size(dims, DSA_WS_LAYER) exceeds
+ *    DSA_NOALLOC_SCRATCH_BYTES return DSA_ERR_SCRATCH_LIMIT (e.g. 1,024 queries
+ *    fit up to a ~6K context at top_k 2048; split larger chunks);
+ *  - the first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture;
+ *  - all calls on a device share the array, and it keeps the last call's
+ *    contents: calls that overlap on the GPU (other streams, other threads)
+ *    race on it. Each call clears the status word and scalars it relies on.
+ * device_status (device memory, 4-byte aligned, may be NULL) receives this
+ * call's device status word, asynchronously on `stream`: 0 on success,
+ * 1 a bounded device wait gave up, 2 an index was out of range, 3 an internal
+ * consistency check failed.
+ * Other arguments and errors are those of dsa_prefill_layer. */
+#define DSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+dsa_status dsa_prefill_layer_noalloc(const dsa_dims* dims, const uint16_t* q,
+                                     const uint16_t* latent, const uint16_t* rope,
+                                     const uint16_t* q_idx, const uint16_t* k_idx,
+                                     const float* w_idx, uint16_t* out, float* lse,
+                                     int32_t* idx_out, uint32_t* device_status, void* stream);
 
 /* Synchronizes `stream`, returns the device status word of `workspace`
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_RANGE) and clears it. */

@@ -29,6 +29,8 @@ DSA_ERR_TIMEOUT = -6
 DSA_ERR_CUDA = -7
 DSA_ERR_DEVICE = -8
 DSA_ERR_RANGE = -9
+DSA_ERR_SCRATCH_LIMIT = -10
+DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 DSA_WS_INDEX_SCORES = 0
 DSA_WS_TOPK = 1
@@ -40,7 +42,7 @@ DSA_MAX_CTX = 49152
 
 EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",
-            "dsa_status_string")
+            "dsa_status_string", "dsa_prefill_layer_noalloc")
 
 
 class dsa_dims(ctypes.Structure):
@@ -87,11 +89,12 @@ def library():
     lib.dsa_sparse_attn_prefill.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     lib.dsa_prefill_layer.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]
+    lib.dsa_prefill_layer_noalloc.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.dsa_device_status.argtypes = [_P, _P]
     lib.dsa_status_string.argtypes = [ctypes.c_int32]
     lib.dsa_status_string.restype = ctypes.c_char_p
     for f in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
-              "dsa_prefill_layer", "dsa_device_status"):
+              "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -164,6 +167,14 @@ def dsa_prefill_layer(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_
                                   _p(k_idx), _p(w_idx), _p(out), _p(lse), _p(idx_out),
                                   _p(workspace), _nbytes(workspace, workspace_bytes),
                                   _stream(stream))
+
+
+def dsa_prefill_layer_noalloc(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out,
+                              device_status=None, stream=None) -> int:
+    """The layer on the library's static scratch array (no workspace argument)."""
+    return library().dsa_prefill_layer_noalloc(_dims(dims), _p(q), _p(latent), _p(rope),
+                                               _p(q_idx), _p(k_idx), _p(w_idx), _p(out), _p(lse),
+                                               _p(idx_out), _p(device_status), _stream(stream))
 
 
 def dsa_device_status(workspace, stream=None) -> int:

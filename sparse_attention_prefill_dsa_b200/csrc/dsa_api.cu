@@ -218,6 +218,8 @@ const char* dsa_status_string(dsa_status s) {
     case DSA_ERR_CUDA: return "CUDA runtime or launch error";
     case DSA_ERR_DEVICE: return "current device is not an sm_100 (B200) GPU";
     case DSA_ERR_RANGE: return "a selected index was outside the causal range";
+    case DSA_ERR_SCRATCH_LIMIT:
+      return "the chunk needs more scratch than the no-alloc entry point's static array holds";
     default: return "unknown status";
   }
 }

@@ -61,7 +61,7 @@ def test_dims_struct_layout_matches_header(dsa):
 
 def test_status_codes_and_strings(dsa):
     text = open(HEADER).read()
-    for name, val in re.findall(r"#define (DSA_(?:OK|ERR_[A-Z]+))\s+\(?(-?\d+)\)?", text):
+    for name, val in re.findall(r"#define (DSA_(?:OK|ERR_[A-Z_]+))\s+\(?(-?\d+)\)?", text):
         assert getattr(dsa, name) == int(val), name
         assert dsa.dsa_status_string(int(val))
     assert dsa.dsa_status_string(12345) == "unknown status"
