@@ -337,11 +337,19 @@ def oracle_sample(d, x, n_rows):
     return n_rows / dt, cores, dt
 
 
-def cpu_baseline(d, x, n_rows):
+def sized_rows(d, x, seconds):
+    """Rows of a CPU-oracle sample that takes about `seconds` on this host."""
+    _, _, dt = oracle_sample(d, x, 8)
+    return int(min(d.n_q, max(8, round(8 * seconds / max(dt, 1e-3)))))
+
+
+def cpu_baseline(d, x, n_rows=None, seconds=12.0):
+    if not n_rows:
+        n_rows = sized_rows(d, x, seconds)
     qps, cores, dt = oracle_sample(d, x, n_rows)
     return {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n_rows} query rows spread over the chunk (float64 oracle, "
-                      f"{dt:.1f} s wall)"}
+            "sample": f"{n_rows} of {d.n_q} query rows spread over the chunk, full layer per "
+                      f"row (float64 oracle, {cores} threads, {dt:.1f} s wall)"}
 
 
 def run_reference(args):
@@ -355,7 +363,7 @@ def run_reference(args):
     d = wl.dims
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     x = workloads.generate(d, wl.seed, wl.kind, w_mode)
-    rows_per_step = args.cpu_rows
+    rows_per_step = args.cpu_rows or sized_rows(d, x, 6.0)
     for _ in range(args.warmup):
         oracle_sample(d, x, max(1, rows_per_step // 4))
     times = []
@@ -373,7 +381,8 @@ def run_reference(args):
         "config": {"workload": wl.name, "about": wl.about, "n_q": d.n_q, "ctx_len": d.ctx_len,
                    "top_k": d.top_k},
         "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{rows_per_step} query rows per step"},
+                         "sample": f"{rows_per_step} of {d.n_q} query rows per step, full "
+                                   f"layer per row (float64 oracle, {cores} threads)"},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -387,8 +396,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="chunk8k_ctx17k", choices=sorted(workloads.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
-    ap.add_argument("--cpu-rows", type=int, default=48,
-                    help="query rows of the bounded CPU-oracle sample")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="query rows of the bounded CPU-oracle sample (0: about 12 s of work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
