@@ -1,81 +1,336 @@
-// indexer.cu -- lightning-indexer scores (component-table row "DSA indexer" of
-// the feedman.me post feedman.me/posts/wy2HU).
+// indexer.cu -- lightning-indexer scores on tcgen05 tensor cores (component-
+// table row "DSA indexer" of the feedman.me post feedman.me/posts/wy2HU).
 //
 //   I[i,s] = sum_j w[i,j] * ReLU( sum_c qI[i,j,c] * kI[s,c] ),  s <= t = q_pos0 + i
 //
-// Straightforward CUDA-core version: a CTA takes 4 queries x 128 keys, stages
-// the queries' indexer rows and the key tile (transposed) in shared memory as
-// float32 and accumulates each head's dot product with sequential float32 FMAs
-// (error <= 128 * 2^-24 * sum|q*k|, inside the selection's 2^-14 bound).
-// Key tiles entirely above the causal boundary are skipped.
+// The head dot products form one dense GEMM per (query block, key tile):
+//   D[s, (i,j)] = sum_c kI[s,c] * qI[i,j,c]
+// with the 128 keys of a tile as the MMA's M dimension and 256 / H_I queries x
+// H_I heads (= 256 columns, query-major, the natural layout of q_idx) as N,
+// K = D_I. Putting keys on M leaves each key's whole row of head dots in one
+// TMEM lane, so the epilogue thread that owns that lane forms ReLU, the
+// w-weighted head sum and the store with no cross-thread traffic, and a warp
+// writes 32 consecutive keys of a query row (128 coalesced bytes).
+//
+// Persistent, warp-specialised CTA (one per SM, 320 threads):
+//   warp 0      TMA producer: the block's q_idx rows (once per work unit) and
+//               a 4-stage ring of key tiles, 128-byte (or 64-byte) swizzled,
+//               plus the block's head weights into a double-buffered slot;
+//   warp 1      TMEM owner and single-thread MMA issuer (tcgen05.mma kind::f16,
+//               bf16 x bf16 -> f32), accumulating each tile into one of two
+//               256-column TMEM buffers;
+//   warps 2-9   epilogue: two warpgroups split the 256 columns; each thread
+//               reads its key's columns with tcgen05.ld and writes the scores.
+// A work unit is (query block, up to 32 consecutive causal key tiles); CTAs
+// take units round-robin. Key tiles past the last query of a block are never
+// loaded (causal skip); rows of a partial tile past the context read as zero
+// and no score past t is written.
+// Every wait is bounded: on a timeout the CTA records DSA_ERR_TIMEOUT in the
+// workspace, all roles stop, outstanding TMA loads and MMAs are drained, and
+// TMEM is freed before the CTA exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "dsa_internal.cuh"
+#include "sm100_primitives.cuh"
 
 namespace dsa {
 namespace {
 
-constexpr int kKeys = 128;  // keys per CTA (one per thread)
-constexpr int kQB = 4;      // queries per CTA
+using namespace sm100;
 
 template <int HI, int DI>
-__global__ void __launch_bounds__(kKeys) index_scores_simple(
-    const uint16_t* __restrict__ q_idx, const uint16_t* __restrict__ k_idx,
-    const float* __restrict__ w_idx, float* __restrict__ scores, int64_t ld, int n_q,
-    int q_pos0) {
-  extern __shared__ __align__(16) float sm[];
-  float* qf = sm;                            // [kQB][HI][DI]
-  float* kT = qf + kQB * HI * DI;            // [DI][kKeys]
-  float* ws = kT + DI * kKeys;               // [kQB][HI]
-  const int i0 = blockIdx.y * kQB;
-  const int s0 = blockIdx.x * kKeys;
-  const int t_max = q_pos0 + min(i0 + kQB, n_q) - 1;
-  if (s0 > t_max) return;  // whole tile is masked for every query of the block
+struct IdxCfg {
+  static constexpr int kM = 128;                       // keys per tile (MMA M)
+  static constexpr int kN = 256;                       // (query, head) columns (MMA N)
+  static constexpr int kQB = kN / HI;                  // queries per block
+  static constexpr int kChunk = DI < 64 ? DI : 64;     // elements per swizzled row
+  static constexpr int kNChunk = DI / kChunk;
+  static constexpr int kRowBytes = kChunk * 2;         // 128 or 64
+  static constexpr uint32_t kSwzCode = kRowBytes == 128 ? 2u : 4u;
+  static constexpr CUtensorMapSwizzle kSwzMap =
+      kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  static constexpr int kSbo = 8 * kRowBytes;           // bytes between 8-row groups
+  static constexpr int kKChunkBytes = kM * kRowBytes;
+  static constexpr int kQChunkBytes = kN * kRowBytes;
+  static constexpr int kKTileBytes = kKChunkBytes * kNChunk;
+  static constexpr int kQBytes = kQChunkBytes * kNChunk;
+  static constexpr int kStages = 4;
+  static constexpr int kKSteps = DI / 16;
+  static constexpr int kStepsPerChunk = kChunk / 16;
+  static constexpr int kTilesPerUnit = 32;
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(kM, kN, false, false);
+  // shared memory carve (offsets from a 1024-byte aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffW = kOffK + kStages * kKTileBytes;        // 2 x 256 floats
+  static constexpr int kOffBar = kOffW + 2 * kN * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
+  static_assert(DI % 16 == 0 && kN % HI == 0 && HI <= 32 && 32 % HI == 0, "shape");
+};
 
-  for (int e = threadIdx.x; e < kQB * HI * DI; e += kKeys) {
-    const int qi = e / (HI * DI);
-    qf[e] = (i0 + qi < n_q) ? bf16_to_f32(q_idx[static_cast<int64_t>(i0) * HI * DI + e]) : 0.f;
-  }
-  for (int e = threadIdx.x; e < kQB * HI; e += kKeys) {
-    const int qi = e / HI;
-    ws[e] = (i0 + qi < n_q) ? w_idx[static_cast<int64_t>(i0) * HI + e] : 0.f;
-  }
-  for (int e = threadIdx.x; e < kKeys * DI; e += kKeys) {
-    const int key = e / DI, c = e - key * DI;
-    const int s = s0 + key;
-    kT[c * kKeys + key] = (s <= t_max) ? bf16_to_f32(k_idx[static_cast<int64_t>(s) * DI + c]) : 0.f;
-  }
-  __syncthreads();
+struct IdxParams {
+  const float* w_idx;
+  float* scores;
+  int64_t ld;
+  int n_q, q_pos0;
+  int n_units, units_per_qb;
+  WsHeader* ws;
+};
 
-  const int s = s0 + threadIdx.x;
-  for (int qi = 0; qi < kQB; ++qi) {
-    const int i = i0 + qi;
-    if (i >= n_q) break;
-    const int t = q_pos0 + i;
-    if (s > t) continue;
-    float acc = 0.f;
-    for (int j = 0; j < HI; ++j) {
-      const float* q = qf + (qi * HI + j) * DI;
-      float dot = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < DI; ++c) dot = fmaf(q[c], kT[c * kKeys + threadIdx.x], dot);
-      acc = fmaf(ws[qi * HI + j], fmaxf(dot, 0.f), acc);
+template <class C>
+__device__ __forceinline__ bool unit_range(const IdxParams& p, int u, int& qb, int& kt0,
+                                           int& kt1) {
+  qb = u / p.units_per_qb;
+  const int c = u - qb * p.units_per_qb;
+  const int last_q = min((qb + 1) * C::kQB, p.n_q) - 1;
+  const int ntiles = (p.q_pos0 + last_q) / C::kM + 1;
+  kt0 = c * C::kTilesPerUnit;
+  kt1 = min(kt0 + C::kTilesPerUnit, ntiles);
+  return kt0 < kt1;
+}
+
+// Wait without the abort shortcut, used only to drain in-flight work.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitLimitCycles) break;
+}
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
+    index_scores_tc(const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_q, const IdxParams p) {
+  using C = IdxCfg<HI, DI>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sQ = smem + C::kOffQ;
+  unsigned char* sK = smem + C::kOffK;
+  float* sW = reinterpret_cast<float*>(smem + C::kOffW);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + C::kStages;
+  uint64_t* q_full = bars + 2 * C::kStages;       // [1]
+  uint64_t* q_empty = q_full + 1;                 // [1]
+  uint64_t* acc_full = q_empty + 1;               // [2]
+  uint64_t* acc_empty = acc_full + 2;             // [2]
+  uint64_t* w_full = acc_empty + 2;               // [2]
+  uint64_t* w_empty = w_full + 2;                 // [2]
+  uint64_t* mma_done = w_empty + 2;               // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
     }
-    scores[static_cast<int64_t>(i) * ld + s] = acc;
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+      mbar_init(&w_full[b], 32);
+      mbar_init(&w_empty[b], 8);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_q);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t it = 0, uq = 0;
+    int q_parity_issued = -1;  // parity of the last q_full phase with copies in flight
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      int qb, kt0, kt1;
+      if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+      // head weights of the block -> sW[uq & 1] (all 32 lanes write and arrive)
+      const int wb = uq & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&w_empty[wb], ((uq >> 1) & 1) ^ 1, abort_flag, p.ws, 1));
+      if (!ok) break;
+      for (int e = lane; e < C::kN; e += 32) {
+        const int i = qb * C::kQB + e / HI;
+        sW[wb * C::kN + e] = i < p.n_q ? __ldg(p.w_idx + static_cast<int64_t>(qb) * C::kN + e) : 0.f;
+      }
+      mbar_arrive(&w_full[wb]);
+      // the block's q_idx rows
+      ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (uq & 1) ^ 1, abort_flag, p.ws, 2));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
+        for (int c = 0; c < C::kNChunk; ++c)
+          tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * C::kChunk, qb * C::kN, q_full);
+      }
+      q_parity_issued = static_cast<int>(uq & 1);
+      for (int kt = kt0; kt < kt1; ++kt, ++it) {
+        const int st = it % C::kStages;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&k_empty[st], ((it / C::kStages) & 1) ^ 1, abort_flag, p.ws, 3));
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&k_full[st], C::kKTileBytes);
+          for (int c = 0; c < C::kNChunk; ++c)
+            tma_load_2d(sK + st * C::kKTileBytes + c * C::kKChunkBytes, &tm_k, c * C::kChunk,
+                        kt * C::kM, &k_full[st]);
+        }
+      }
+      if (ok) ++uq;
+    }
+    if (!ok && lane == 0) {  // let every issued copy land before the CTA exits
+      const uint32_t n_back = it < static_cast<uint32_t>(C::kStages) ? it : C::kStages;
+      for (uint32_t b = 1; b <= n_back; ++b) {
+        const uint32_t tile = it - b;
+        drain_wait(&k_full[tile % C::kStages], (tile / C::kStages) & 1);
+      }
+      if (q_parity_issued >= 0) drain_wait(q_full, static_cast<uint32_t>(q_parity_issued));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, uq = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int qb, kt0, kt1;
+        if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+        if (!(ok = mbar_wait(q_full, uq & 1, abort_flag, p.ws, 4))) break;
+        for (int kt = kt0; kt < kt1; ++kt, ++it) {
+          const int st = it % C::kStages, buf = it & 1;
+          if (!(ok = mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, abort_flag, p.ws, 5))) break;
+          if (!(ok = mbar_wait(&k_full[st], (it / C::kStages) & 1, abort_flag, p.ws, 6))) break;
+          tc_fence_after();
+          const uint32_t d = tmem_base + buf * C::kN;
+          const uint32_t k_addr = smem_u32(sK + st * C::kKTileBytes);
+          const uint32_t q_addr = smem_u32(sQ);
+#pragma unroll
+          for (int ks = 0; ks < C::kKSteps; ++ks) {
+            const int c = ks / C::kStepsPerChunk;
+            const uint32_t off = (ks % C::kStepsPerChunk) * 32;
+            const uint64_t a = smem_desc(k_addr + c * C::kKChunkBytes + off, 16, C::kSbo, C::kSwzCode);
+            const uint64_t b = smem_desc(q_addr + c * C::kQChunkBytes + off, 16, C::kSbo, C::kSwzCode);
+            mma_bf16_ss(d, a, b, C::kIdesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&k_empty[st]);
+          mma_commit(&acc_full[buf]);
+        }
+        if (!ok) break;
+        mma_commit(q_empty);
+        ++uq;
+      }
+      // every MMA issued must complete before TMEM is released
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int wg = (warp - 2) >> 2;        // column half
+    const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+    const int key_local = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t it = 0, uq = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      int qb, kt0, kt1;
+      if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+      const int wb = uq & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&w_full[wb], (uq >> 1) & 1, abort_flag, p.ws, 7));
+      if (!ok) break;
+      const float* w = sW + wb * C::kN;
+      for (int kt = kt0; kt < kt1; ++kt, ++it) {
+        const int buf = it & 1;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&acc_full[buf], (it >> 1) & 1, abort_flag, p.ws, 8));
+        if (!ok) break;
+        tc_fence_after();
+        const int s = kt * C::kM + key_local;
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+          const int col0 = wg * 128 + g * 32;
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + col0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int qq = 0; qq < 32 / HI; ++qq) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < HI; ++j)
+              acc = fmaf(w[col0 + qq * HI + j], fmaxf(__uint_as_float(v[qq * HI + j]), 0.f), acc);
+            const int i = qb * C::kQB + (col0 + qq * HI) / HI;
+            if (i < p.n_q && s <= p.q_pos0 + i) p.scores[static_cast<int64_t>(i) * p.ld + s] = acc;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&w_empty[wb]);
+      ++uq;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+constexpr int kOneCtaPerSmSmem = 120 * 1024;
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 template <int HI, int DI>
 cudaError_t launch(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_idx,
-                   const float* w_idx, float* scores, int64_t ld, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (kQB * HI * DI + DI * kKeys + kQB * HI);
-  cudaFuncSetAttribute(index_scores_simple<HI, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(smem));
-  const int T_used = d.q_pos0 + d.n_q;
-  dim3 grid((T_used + kKeys - 1) / kKeys, (d.n_q + kQB - 1) / kQB);
-  index_scores_simple<HI, DI><<<grid, kKeys, smem, st>>>(q_idx, k_idx, w_idx, scores, ld, d.n_q,
-                                                         d.q_pos0);
+                   const float* w_idx, float* scores, int64_t ld, WsHeader* ws, cudaStream_t st) {
+  using C = IdxCfg<HI, DI>;
+  CUtensorMap tm_k, tm_q;
+  if (!make_tmap_bf16_2d(&tm_k, k_idx, DI, static_cast<uint64_t>(d.ctx_len), C::kChunk, C::kM,
+                         C::kSwzMap) ||
+      !make_tmap_bf16_2d(&tm_q, q_idx, DI, static_cast<uint64_t>(d.n_q) * HI, C::kChunk, C::kN,
+                         C::kSwzMap))
+    return cudaErrorInvalidValue;
+  IdxParams p;
+  p.w_idx = w_idx;
+  p.scores = scores;
+  p.ld = ld;
+  p.n_q = d.n_q;
+  p.q_pos0 = d.q_pos0;
+  p.ws = ws;
+  const int max_tiles = (d.q_pos0 + d.n_q - 1) / C::kM + 1;
+  p.units_per_qb = (max_tiles + C::kTilesPerUnit - 1) / C::kTilesPerUnit;
+  const int n_qb = (d.n_q + C::kQB - 1) / C::kQB;
+  p.n_units = n_qb * p.units_per_qb;
+  const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
+  // The CTA owns all 512 TMEM columns of its SM: ask for enough shared memory
+  // that a second CTA can never be resident beside it.
+  const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
+  cudaError_t e = cudaFuncSetAttribute(index_scores_tc<HI, DI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  index_scores_tc<HI, DI><<<grid, C::kThreads, smem, st>>>(tm_k, tm_q, p);
   return cudaGetLastError();
 }
 
@@ -84,11 +339,10 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_i
 cudaError_t launch_index_scores(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_idx,
                                 const float* w_idx, float* scores, int64_t ld, WsHeader* ws,
                                 cudaStream_t st) {
-  (void)ws;
   if (d.n_idx_heads == 32 && d.d_idx == 128)
-    return launch<32, 128>(d, q_idx, k_idx, w_idx, scores, ld, st);
+    return launch<32, 128>(d, q_idx, k_idx, w_idx, scores, ld, ws, st);
   if (d.n_idx_heads == 2 && d.d_idx == 32)
-    return launch<2, 32>(d, q_idx, k_idx, w_idx, scores, ld, st);
+    return launch<2, 32>(d, q_idx, k_idx, w_idx, scores, ld, ws, st);
   return cudaErrorInvalidValue;
 }
 
