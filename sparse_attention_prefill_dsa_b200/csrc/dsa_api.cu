@@ -158,7 +158,7 @@ dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const u
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = clear_header(ws, st)) != DSA_OK) return s;
   if (d->n_q == 0) return DSA_OK;
-  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse,
+  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, false,
                                            static_cast<WsHeader*>(ws), st));
 }
 
@@ -189,7 +189,7 @@ dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   e = dsa::launch_topk(*d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
-  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, h, st));
+  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, true, h, st));
 }
 
 dsa_status dsa_device_status(void* ws, void* stream) {

@@ -52,8 +52,10 @@ cudaError_t launch_key_norm_max(const dsa_dims& d, const uint16_t* k_idx, WsHead
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld,
                         const uint16_t* q_idx, const uint16_t* k_idx, const float* w_idx,
                         int32_t* idx, WsHeader* ws, cudaStream_t st);
+// prefix_valid: every idx row holds its min(top_k, t+1) valid keys first (as the
+// selections of dsa_topk_select do), so tiles past them are skipped.
 cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,
-                               float* lse, WsHeader* ws, cudaStream_t st);
+                               float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st);
 
 }  // namespace dsa
