@@ -16,7 +16,8 @@
 // Per query, in tiles of 128 selected keys:
 //   gather   latent (8 x 64-dim chunks) and rope rows of the tile into nine
 //            16 KB shared-memory slots, 128-byte swizzled, one key per 128-byte
-//            row (cp.async, four producer warps);
+//            row (cp.async, four producer warps; each slot's mbarrier completes
+//            when its copies land, via cp.async.mbarrier.arrive.noinc);
 //   QK^T     S^T[key, head] = K_tile . Q^T: keys are the MMA's M (128), the
 //            padded heads its N, K = Dc + Dr, both operands K-major; rope
 //            chunk first so its slot is released earliest;
@@ -242,29 +243,13 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     // issues the next one; before any wait that could block, pending copies
     // are completed and announced, so the producer never holds back data a
     // consumer needs to make progress.
-    uint64_t* pending = nullptr;
-    auto announce_pending = [&]() {
-      if (pending) {
-        cp_async_wait_group<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(pending);
-        pending = nullptr;
-      }
-    };
+    // Each lane announces its copies with cp.async.mbarrier.arrive.noinc: the
+    // barrier completes when the copies have landed, so a producer never
+    // waits on its own copies and never holds data a consumer needs.
     auto wait_free = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
-      if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-      announce_pending();
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.ws, site));
     };
-    auto issued = [&](uint64_t* bar) {
-      cp_async_commit();
-      if (pending) {
-        cp_async_wait_group<1>();
-        fence_proxy_async_smem();
-        mbar_arrive(pending);
-      }
-      pending = bar;
-    };
+    auto issued = [&](uint64_t* bar) { cp_async_arrive_noinc(bar); };
     uint32_t tc = 0, qi = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
@@ -281,38 +266,50 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       issued(q_full);
       const int nt = n_tiles_of(p, i);
       const int32_t* irow = p.idx + static_cast<int64_t>(i) * p.k;
+      const int part = lane & 7;
       for (int j = 0; j < nt && ok; ++j, ++tc) {
+        // the 32 cache rows this lane copies in every slot of the tile:
+        // keys (lane >> 3) + 4 * it, loaded up front with independent loads
+        int rows[32];
+#pragma unroll
+        for (int it = 0; it < 32; ++it) {
+          const int sel = j * 128 + (lane >> 3) + 4 * it;
+          rows[it] = sel < p.k ? __ldg(irow + sel) : -1;
+        }
+#pragma unroll
+        for (int it = 0; it < 32; ++it) {
+          if (rows[it] >= p.ctx_len) {
+            report(p.ws, kDevRange, static_cast<unsigned>(i));
+            rows[it] = -1;
+          }
+          if (rows[it] < 0) rows[it] = 0;  // masked key: any finite row; its weight is zero
+        }
         for (int pos = warp; pos < C::kGatherPositions; pos += 4) {
           const int slot = pos == 0 ? C::kRope : pos - 1;
           if (!(ok = wait_free(&slot_empty[slot], (tc & 1) ^ 1, 21))) break;
           unsigned char* dst = sSlots + slot * C::kSlotBytes;
-          const int part = lane & 7;
-          if (slot != C::kRope || part < DR / 8) {
-#pragma unroll 4
+          if (slot == C::kRope) {
+            if (part < DR / 8) {
+#pragma unroll
+              for (int it = 0; it < 32; ++it) {
+                const int key = (lane >> 3) + 4 * it;
+                cp_async_16(dst + key * 128 + ((part ^ (key & 7)) << 4),
+                            p.rope + static_cast<int64_t>(rows[it]) * DR + part * 8);
+              }
+            }
+          } else {
+#pragma unroll
             for (int it = 0; it < 32; ++it) {
               const int key = (lane >> 3) + 4 * it;
-              const int sel = j * 128 + key;
-              int row = sel < p.k ? __ldg(irow + sel) : -1;
-              if (row >= p.ctx_len) {
-                report(p.ws, kDevRange, static_cast<unsigned>(i));
-                row = -1;
-              }
-              if (row < 0) row = 0;  // masked key: any finite row; its weight is zero
-              const uint16_t* src = slot == C::kRope
-                                        ? p.rope + static_cast<int64_t>(row) * DR + part * 8
-                                        : p.latent + static_cast<int64_t>(row) * DC + slot * 64 + part * 8;
-              cp_async_16(dst + key * 128 + ((part ^ (key & 7)) << 4), src);
+              cp_async_16(dst + key * 128 + ((part ^ (key & 7)) << 4),
+                          p.latent + static_cast<int64_t>(rows[it]) * DC + slot * 64 + part * 8);
             }
           }
           issued(&slot_full[slot]);
         }
       }
     }
-    if (ok) {
-      announce_pending();
-    } else {
-      cp_async_wait_group<0>();  // let every copy land before the CTA exits
-    }
+    cp_async_wait_all();  // every copy lands before the CTA can exit
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -325,12 +322,14 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         const int nt = n_tiles_of(p, i);
         const int ob = qi & 1;
         if (!(ok = mbar_wait(q_full, qi & 1, abort_flag, p.ws, 30))) break;
+        fence_proxy_async_smem();
         for (int j = 0; j < nt; ++j, ++tc) {
           const int sb = tc & 1, pb = tc & 1;
           // ---- S^T = K_tile . Q^T
           if (!(ok = mbar_wait(&s_empty[sb], ((tc >> 1) & 1) ^ 1, abort_flag, p.ws, 31))) break;
           const uint32_t d_s = tmem_base + C::kTmemS + sb * NH;
           if (!(ok = mbar_wait(&slot_full[C::kRope], tc & 1, abort_flag, p.ws, 32))) break;
+          fence_proxy_async_smem();
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < C::kRopeSteps; ++ks) {
@@ -341,6 +340,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           mma_commit(&slot_empty[C::kRope]);
           for (int c = 0; c < C::NL && ok; ++c) {
             if (!(ok = mbar_wait(&slot_full[c], tc & 1, abort_flag, p.ws, 33))) break;
+            fence_proxy_async_smem();
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
@@ -402,6 +402,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       }
       for (int j = 0; j < nt; ++j, ++tc) {
         const int sb = tc & 1, pb = tc & 1;
+        const int sel = j * 128 + r;
+        const int row = sel < p.k ? __ldg(irow + sel) : -1;  // issued before the wait
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (tc >> 1) & 1, abort_flag, p.ws, 40));
         if (!ok) break;
         tc_fence_after();
@@ -409,8 +411,6 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * NH, x);
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
-        const int sel = j * 128 + r;
-        int row = sel < p.k ? __ldg(irow + sel) : -1;
         const bool valid = row >= 0 && row < p.ctx_len;
 #pragma unroll
         for (int h = 0; h < NH; ++h) x[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;

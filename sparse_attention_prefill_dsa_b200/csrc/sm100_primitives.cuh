@@ -192,6 +192,17 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Arrives on `bar` (without raising its expected count) once every cp.async
+// this thread issued so far has landed in shared memory.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Makes this thread's prior generic-proxy shared-memory writes (plain stores
 // and completed cp.async copies) visible to the async proxy (tensor cores).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -106,8 +106,8 @@ def test_index_scores_within_certified_bound(dsa, oracle_lib):
         t = d.q_pos0 + i
         err = np.abs(f32[i, : t + 1].astype(np.float64) - ref[i, : t + 1]).max()
         worst = max(worst, err / (A[i] * kmax))
-    bound = 2.0 ** -14 + 2.0 ** -17
-    print(f"worst |F-X| / (A_t Kmax) = {worst:.3e} (bound {bound:.3e})")
+    bound = 2.0 ** -15 + 2.0 ** -17
+    print(f"\nworst |F-X| / (A_t Kmax) = {worst:.3e} (bound {bound:.3e}, ratio {bound / worst:.0f}x)")
     assert worst <= bound / 16
 
 
