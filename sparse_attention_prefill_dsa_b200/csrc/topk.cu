@@ -129,22 +129,24 @@ __device__ __forceinline__ unsigned long long block_excl_scan64(unsigned long lo
   return base + x - v;
 }
 
-// hist[0..kBins) counts; finds bin b with sum(hist[b+1..]) < kr <= sum(hist[b..]).
+// hist[0..NB) counts; finds bin b with sum(hist[b+1..]) < kr <= sum(hist[b..]).
+template <int NB>
 __device__ int find_bin_from_top(const int* hist, int kr, int* above, Scratch& sc) {
-  constexpr int per = kBins / kThreads;  // 8 bins per thread, counted from the top
+  constexpr int per = (NB + kThreads - 1) / kThreads;  // bins per thread, counted from the top
   const int r0 = threadIdx.x * per;
   int local = 0;
 #pragma unroll
-  for (int e = 0; e < per; ++e) local += hist[kBins - 1 - (r0 + e)];
+  for (int e = 0; e < per; ++e)
+    if (r0 + e < NB) local += hist[NB - 1 - (r0 + e)];
   unsigned long long tot;
   const int before =
       static_cast<int>(block_excl_scan64(static_cast<unsigned long long>(local), &tot, sc));
   if (before < kr && before + local >= kr) {
     int acc = before;
-    for (int e = 0; e < per; ++e) {
-      const int c = hist[kBins - 1 - (r0 + e)];
+    for (int e = 0; e < per && r0 + e < NB; ++e) {
+      const int c = hist[NB - 1 - (r0 + e)];
       if (acc + c >= kr) {
-        sc.bc[0] = kBins - 1 - (r0 + e);
+        sc.bc[0] = NB - 1 - (r0 + e);
         sc.bc[1] = acc;
         break;
       }
@@ -167,10 +169,30 @@ __device__ __forceinline__ void my_segment(int n, int& beg, int& end) {
   end = min(beg + len, n);
 }
 
-__device__ __forceinline__ int bucket_of(float v, double L, double scale) {
-  const double x = (static_cast<double>(v) - L) * scale;
-  return x >= static_cast<double>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
-}
+// Bucket of v in [L, U]: floor((v - L) * scale), clamped to the last bucket.
+// Rounded float arithmetic is monotone in v, which is all the select needs;
+// ranges too narrow for a finite float scale use float64.
+struct Bucketer {
+  float Lf, scalef;
+  double Ld, scaled;
+  bool wide;
+  __device__ __forceinline__ Bucketer(float L, float U) {
+    const float range = U - L;
+    wide = range > 1e-30f && range < 1e30f;
+    Lf = L;
+    scalef = wide ? static_cast<float>(kBins) / range : 0.f;
+    Ld = L;
+    scaled = static_cast<double>(kBins) / (static_cast<double>(U) - static_cast<double>(L));
+  }
+  __device__ __forceinline__ int operator()(float v) const {
+    if (wide) {
+      const float x = (v - Lf) * scalef;
+      return x >= static_cast<float>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
+    }
+    const double x = (static_cast<double>(v) - Ld) * scaled;
+    return x >= static_cast<double>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
+  }
+};
 
 // Exact k-th largest of sc[0..n) (n > k). *n_above gets the number of values
 // strictly larger. Uses hist[kBins] and cand[kCandCap]. Returns false if the
@@ -190,21 +212,21 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
     for (int b = threadIdx.x; b < kBins; b += kThreads) hist[b] = 0;
     if (threadIdx.x == 0) sm.bc[2] = 0;
     __syncthreads();
-    const double Ld = L, scale = static_cast<double>(kBins) / (static_cast<double>(U) - Ld);
+    const Bucketer bucket(L, U);
     for (int s = beg; s < end; ++s) {
       const float v = sc[s];
-      if (v >= L && v <= U) atomicAdd(&hist[bucket_of(v, Ld, scale)], 1);
+      if (v >= L && v <= U) atomicAdd(&hist[bucket(v)], 1);
     }
     __syncthreads();
     int ab;
-    const int bstar = find_bin_from_top(hist, kr, &ab, sm);
+    const int bstar = find_bin_from_top<kBins>(hist, kr, &ab, sm);
     kr -= ab;
     above += ab;
     const int c = hist[bstar];
     float mn = INFINITY, mx = -INFINITY;
     for (int s = beg; s < end; ++s) {
       const float v = sc[s];
-      if (v >= L && v <= U && bucket_of(v, Ld, scale) == bstar) {
+      if (v >= L && v <= U && bucket(v) == bstar) {
         mn = fminf(mn, v);
         mx = fmaxf(mx, v);
         if (c <= kCandCap) cand[atomicAdd(&sm.bc[2], 1)] = v;
@@ -392,7 +414,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   unsigned char* p = reinterpret_cast<unsigned char*>(cand + kCandCap);
   uint16_t* qT = reinterpret_cast<uint16_t*>(p);  p += sizeof(uint16_t) * 32 * 128;
   float* w_s = reinterpret_cast<float*>(p);       p += sizeof(float) * 32;
-  uint16_t* kst = reinterpret_cast<uint16_t*>(p); p += sizeof(uint16_t) * kWarps * 512;
+  uint16_t* kst = reinterpret_cast<uint16_t*>(hist);  // hist/cand are free from here on
   int* tile_s = reinterpret_cast<int*>(p);        p += sizeof(int) * kThreads;
   double* tile_x = reinterpret_cast<double*>(p);  p += sizeof(double) * kThreads;
   unsigned long long* bx = reinterpret_cast<unsigned long long*>(p);
@@ -426,11 +448,19 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
 
   int beg, end;
   my_segment(n, beg, end);
+  // one pass: count the certainly-kept keys and the band, collecting band keys
+  // (any order) while they fit the cache
+  if (threadIdx.x == 0) sm.bc[2] = 0;
+  __syncthreads();
   int c_in = 0, c_band = 0;
   for (int s = beg; s < end; ++s) {
     const double f = sc[s];
     c_in += f > hi;
-    c_band += (f >= lo && f <= hi);
+    if (f >= lo && f <= hi) {
+      ++c_band;
+      const int pos = atomicAdd(&sm.bc[2], 1);
+      if (pos < a.bcap) bidx[pos] = s;
+    }
   }
   unsigned long long tot;
   block_excl_scan64(
@@ -457,15 +487,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   uint16_t* my_kst = kst + warp * 512;
 
   if (tot_band <= a.bcap) {
-    // collect the band (any order), re-score it, rank it by (X desc, index asc),
-    // and mark the row: kept band keys -> +inf, dropped -> -inf
-    if (threadIdx.x == 0) sm.bc[2] = 0;
-    __syncthreads();
-    for (int s = beg; s < end; ++s) {
-      const double f = sc[s];
-      if (f >= lo && f <= hi) bidx[atomicAdd(&sm.bc[2], 1)] = s;
-    }
-    __syncthreads();
+    // re-score the collected band, rank it by (X desc, index asc), and mark
+    // the row: kept band keys -> +inf, dropped -> -inf
     for (int b = 4 * warp; b < tot_band; b += 4 * kWarps) {
       const int nk = min(4, tot_band - b);
       int ks[4];
@@ -532,22 +555,22 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     __syncthreads();
     return nb;
   };
+  int* hist256 = reinterpret_cast<int*>(cand);  // cand is free; hist holds the staging rows
   unsigned long long pre = 0ull, msk = 0ull;
   int rr = r;
   for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < kBins; b += kThreads) hist[b] = 0;
+    for (int b = threadIdx.x; b < 256; b += kThreads) hist256[b] = 0;
     __syncthreads();
     for (int base = 0; base < n; base += kThreads) {
       const int nb = band_window(base);
       if (static_cast<int>(threadIdx.x) < nb) {
         const unsigned long long key = d2key(tile_x[threadIdx.x]);
-        // digits go to the top 256 bins so find_bin_from_top sees them in order
-        if ((key & msk) == pre) atomicAdd(&hist[kBins - 256 + static_cast<int>((key >> shift) & 0xFFull)], 1);
+        if ((key & msk) == pre) atomicAdd(&hist256[static_cast<int>((key >> shift) & 0xFFull)], 1);
       }
       __syncthreads();
     }
     int ab;
-    const int bin = find_bin_from_top(hist, rr, &ab, sm) - (kBins - 256);
+    const int bin = find_bin_from_top<256>(hist256, rr, &ab, sm);
     rr -= ab;
     pre |= static_cast<unsigned long long>(bin) << shift;
     msk |= 0xFFull << shift;
@@ -627,8 +650,8 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   size_t bytes = sizeof(float) * a.n_cap + sizeof(int) * kBins + sizeof(float) * kCandCap;
   a.bcap = 0;
   if (refine) {
-    bytes += sizeof(uint16_t) * 32 * 128 + sizeof(float) * 32 + sizeof(uint16_t) * kWarps * 512 +
-             sizeof(int) * kThreads + sizeof(double) * kThreads;
+    bytes += sizeof(uint16_t) * 32 * 128 + sizeof(float) * 32 + sizeof(int) * kThreads +
+             sizeof(double) * kThreads;
     if (static_cast<size_t>(max_smem) < bytes + static_bytes) return cudaErrorInvalidConfiguration;
     // band cache of up to 1,024 keys; when the row is short enough, sized so
     // that two CTAs still fit on one SM
