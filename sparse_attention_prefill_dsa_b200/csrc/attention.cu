@@ -16,19 +16,21 @@
 // Per query, in tiles of 128 selected keys:
 //   gather   latent (8 x 64-dim chunks) and rope rows of the tile into nine
 //            16 KB shared-memory slots, 128-byte swizzled, one key per 128-byte
-//            row (cp.async, four producer warps; each slot's mbarrier completes
-//            when its copies land, via cp.async.mbarrier.arrive.noinc);
+//            row, with TMA tile::gather4 loads (four selected rows each);
 //   QK^T     S^T[key, head] = K_tile . Q^T: keys are the MMA's M (128), the
 //            padded heads its N, K = Dc + Dr, both operands K-major; rope
-//            chunk first so its slot is released earliest;
+//            chunk first so its slot is released earliest. A tcgen05.mma that
+//            depends on the previous one's accumulator waits out its latency,
+//            so the K steps feed four independent partial sums (summed by the
+//            softmax) and the PV interleaves its four 128-dim output blocks;
 //   softmax  one thread per key lane of S^T: the per-head tile maximum is found
 //            with a warp transpose-reduction plus a four-warp exchange through
 //            shared memory (mbarrier-synchronised), the running maximum is
 //            raised only when a tile exceeds it by more than 2^8 (then O and
 //            the partial sums are rescaled), and p = 2^(z log2e - m) is written
-//            as bf16 into P^T [head, key];
+//            as bf16 into P [key, head] (one 16-byte-chunked row per key);
 //   PV       O^T[dim, head] += latent_tile^T . P^T: the same latent slots read
-//            MN-major as A (dims as M, four 128-dim blocks), P^T K-major as B;
+//            MN-major as A (dims as M, four 128-dim blocks), P MN-major as B;
 //            each block's two slots are released as soon as its MMAs finish,
 //            so the next tile's gather overlaps the current PV.
 // Accumulators live in TMEM (S^T double-buffered per tile, O^T per query);
@@ -40,6 +42,7 @@
 //   warps 5-8  softmax and epilogue (TMEM lanes 0-127 = keys, then dims).
 // Every wait is bounded; on a timeout the CTA records DSA_ERR_TIMEOUT, all
 // roles stop, copies and MMAs in flight are drained and TMEM is freed.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -65,15 +68,22 @@ struct AttnCfg {
   static constexpr int kSlotBytes = kKeys * 128;      // 16 KB
   static constexpr int kQChunks = NL + 1;             // latent chunks + rope chunk
   static constexpr int kQChunkBytes = NH * 128;
-  static constexpr int kPBytes = 2 * NH * 128;        // P^T: NH rows x 128 keys (2 chunks)
+  // P: one row of NH bf16 per key (MN-major B operand of the PV), 64- or
+  // 32-byte rows swizzled in 8-row atoms
+  static constexpr int kPRowBytes = NH * 2;
+  static constexpr int kPBytes = kKeys * kPRowBytes;
+  static constexpr uint32_t kPSwz = NH == 32 ? 4u : 6u;  // descriptor code: 64B / 32B swizzle
   static constexpr int kThreads = 288;
   static constexpr int kGatherPositions = NL + 1;     // rope, L0..L(NL-1)
+  static constexpr bool kRopeTma = DR == 64;          // a 128-byte rope row: TMA gather4
+  static constexpr uint32_t kQBytes = H * 128 * kQChunks;  // q boxes (zero-filled past Dc+Dr)
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, NH, false, false);
-  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, NH, true, false);
-  // TMEM columns: S^T[2] then O^T[2][MB]
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, NH, true, true);
+  // TMEM columns: S^T[2 buffers][kChains partial sums] then O^T[2][MB]
+  static constexpr int kChains = 4;                   // independent QK^T accumulators
   static constexpr int kTmemS = 0;
-  static constexpr int kTmemO = 2 * NH;
-  static constexpr int kTmemUsed = 2 * NH + 2 * MB * NH;
+  static constexpr int kTmemO = 2 * kChains * NH;
+  static constexpr int kTmemUsed = 2 * kChains * NH + 2 * MB * NH;
   static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
   // shared memory carve (from a 1024-byte aligned base)
@@ -175,7 +185,8 @@ __device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&x)[NH]
 
 template <int H, int DC, int DR>
 __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
-    sparse_attn_tc(const AttnParams p) {
+    sparse_attn_tc(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
+                   const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
   using C = AttnCfg<H, DC, DR>;
   constexpr int NH = C::NH;
   extern __shared__ unsigned char smem_raw[];
@@ -211,10 +222,12 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kSlots; ++s) {
-      mbar_init(&slot_full[s], 32);
+      // TMA slots complete on bytes after one arrive; a cp.async rope slot on
+      // the 32 noinc arrivals of its warp
+      mbar_init(&slot_full[s], (s == C::kRope && !C::kRopeTma) ? 32 : 1);
       mbar_init(&slot_empty[s], 1);
     }
-    mbar_init(q_full, 128);
+    mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -238,78 +251,91 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
   if (warp < 4) {
     // -------------------------------------------------------------- producers
     // This warp fills gather positions w, w+4, ... of each tile (position 0 is
-    // the rope chunk, position 1+c latent chunk c) and q chunks w, w+4, ...
-    // (chunk NL is the rope part). A copy group stays pending while the warp
-    // issues the next one; before any wait that could block, pending copies
-    // are completed and announced, so the producer never holds back data a
-    // consumer needs to make progress.
-    // Each lane announces its copies with cp.async.mbarrier.arrive.noinc: the
-    // barrier completes when the copies have landed, so a producer never
-    // waits on its own copies and never holds data a consumer needs.
-    auto wait_free = [&](uint64_t* bar, uint32_t parity, unsigned site) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.ws, site));
-    };
-    auto issued = [&](uint64_t* bar) { cp_async_arrive_noinc(bar); };
+    // the rope chunk, position 1+c latent chunk c). A slot of 128 keys is 32
+    // TMA gather4 loads, one per lane: lane l brings keys 4l..4l+3 (four
+    // 128-byte rows, 512 swizzled bytes) and the slot's mbarrier completes on
+    // its 16 KB of transactions. Warp 0 also loads the query's q rows with 2D
+    // TMA boxes. A 16-dim rope chunk (too narrow for a 128-byte swizzled box)
+    // is gathered with cp.async, each lane announcing its copies with
+    // cp.async.mbarrier.arrive.noinc.
+    if (warp == 0 && lane == 0) {
+      prefetch_tmap(&tm_lat);
+      prefetch_tmap(&tm_q);
+      if (C::kRopeTma) prefetch_tmap(&tm_rope);
+    }
     uint32_t tc = 0, qi = 0;
     bool ok = true;
+    int last_slot_parity = -1;  // parity of this warp's last issued slot fills (for draining)
+    int q_parity = -1;
     for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
-      // q rows of this query
-      if (!(ok = wait_free(q_empty, (qi & 1) ^ 1, 20))) break;
-      for (int c = warp; c < C::kQChunks; c += 4) {
-        const int parts = c < C::NL ? 8 : DR / 8;
-        for (int e = lane; e < H * parts; e += 32) {
-          const int h = e / parts, part = e - h * parts;
-          const uint16_t* src = p.q + (static_cast<int64_t>(i) * H + h) * (DC + DR) + c * 64 + part * 8;
-          cp_async_16(sQ + c * C::kQChunkBytes + h * 128 + ((part ^ (h & 7)) << 4), src);
+      if (warp == 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (qi & 1) ^ 1, abort_flag, p.ws, 20));
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, C::kQBytes);
+          for (int c = 0; c < C::kQChunks; ++c)
+            tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, i * H, q_full);
         }
+        q_parity = qi & 1;
       }
-      issued(q_full);
       const int nt = n_tiles_of(p, i);
       const int32_t* irow = p.idx + static_cast<int64_t>(i) * p.k;
-      const int part = lane & 7;
       for (int j = 0; j < nt && ok; ++j, ++tc) {
-        // the 32 cache rows this lane copies in every slot of the tile:
-        // keys (lane >> 3) + 4 * it, loaded up front with independent loads
-        int rows[32];
+        // rows of keys 4*lane .. 4*lane+3 (masked or out-of-range keys read row 0;
+        // their softmax weight is zero)
+        int r4[4];
 #pragma unroll
-        for (int it = 0; it < 32; ++it) {
-          const int sel = j * 128 + (lane >> 3) + 4 * it;
-          rows[it] = sel < p.k ? __ldg(irow + sel) : -1;
-        }
-#pragma unroll
-        for (int it = 0; it < 32; ++it) {
-          if (rows[it] >= p.ctx_len) {
+        for (int e = 0; e < 4; ++e) {
+          const int sel = j * 128 + 4 * lane + e;
+          int row = sel < p.k ? __ldg(irow + sel) : -1;
+          if (row >= p.ctx_len) {
             report(p.ws, kDevRange, static_cast<unsigned>(i));
-            rows[it] = -1;
+            row = -1;
           }
-          if (rows[it] < 0) rows[it] = 0;  // masked key: any finite row; its weight is zero
+          r4[e] = row < 0 ? 0 : row;
         }
         for (int pos = warp; pos < C::kGatherPositions; pos += 4) {
           const int slot = pos == 0 ? C::kRope : pos - 1;
-          if (!(ok = wait_free(&slot_empty[slot], (tc & 1) ^ 1, 21))) break;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&slot_empty[slot], (tc & 1) ^ 1, abort_flag, p.ws, 21));
+          if (!ok) break;
           unsigned char* dst = sSlots + slot * C::kSlotBytes;
-          if (slot == C::kRope) {
+          if (slot != C::kRope || C::kRopeTma) {
+            if (lane == 0) mbar_arrive_expect_tx(&slot_full[slot], C::kSlotBytes);
+            __syncwarp();
+            if (slot == C::kRope)
+              tma_gather4(dst + lane * 512, &tm_rope, 0, r4[0], r4[1], r4[2], r4[3], &slot_full[slot]);
+            else
+              tma_gather4(dst + lane * 512, &tm_lat, slot * 64, r4[0], r4[1], r4[2], r4[3],
+                          &slot_full[slot]);
+          } else {
+            const int part = lane & 7;
             if (part < DR / 8) {
-#pragma unroll
+#pragma unroll 4
               for (int it = 0; it < 32; ++it) {
                 const int key = (lane >> 3) + 4 * it;
+                const int sel = j * 128 + key;
+                int row = sel < p.k ? __ldg(irow + sel) : -1;
+                if (row < 0 || row >= p.ctx_len) row = 0;
                 cp_async_16(dst + key * 128 + ((part ^ (key & 7)) << 4),
-                            p.rope + static_cast<int64_t>(rows[it]) * DR + part * 8);
+                            p.rope + static_cast<int64_t>(row) * DR + part * 8);
               }
             }
-          } else {
-#pragma unroll
-            for (int it = 0; it < 32; ++it) {
-              const int key = (lane >> 3) + 4 * it;
-              cp_async_16(dst + key * 128 + ((part ^ (key & 7)) << 4),
-                          p.latent + static_cast<int64_t>(rows[it]) * DC + slot * 64 + part * 8);
-            }
+            cp_async_arrive_noinc(&slot_full[slot]);
           }
-          issued(&slot_full[slot]);
+          last_slot_parity = tc & 1;
         }
       }
     }
-    cp_async_wait_all();  // every copy lands before the CTA can exit
+    cp_async_wait_all();  // every cp.async copy lands before the CTA can exit
+    if (!ok && lane == 0) {  // and every TMA load this warp issued
+      if (last_slot_parity >= 0)
+        for (int pos = warp; pos < C::kGatherPositions; pos += 4) {
+          const int slot = pos == 0 ? C::kRope : pos - 1;
+          if (slot != C::kRope || C::kRopeTma) drain_wait(&slot_full[slot], last_slot_parity);
+        }
+      if (q_parity >= 0) drain_wait(q_full, q_parity);
+    }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -327,7 +353,10 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           const int sb = tc & 1, pb = tc & 1;
           // ---- S^T = K_tile . Q^T
           if (!(ok = mbar_wait(&s_empty[sb], ((tc >> 1) & 1) ^ 1, abort_flag, p.ws, 31))) break;
-          const uint32_t d_s = tmem_base + C::kTmemS + sb * NH;
+          // S^T accumulates in kChains independent partial sums (K-step ks of
+          // every chunk goes to chain ks), so consecutive MMAs never wait on
+          // each other's accumulator; the softmax adds the partials.
+          const uint32_t d_s = tmem_base + C::kTmemS + sb * C::kChains * NH;
           if (!(ok = mbar_wait(&slot_full[C::kRope], tc & 1, abort_flag, p.ws, 32))) break;
           fence_proxy_async_smem();
           tc_fence_after();
@@ -335,7 +364,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           for (int ks = 0; ks < C::kRopeSteps; ++ks) {
             const uint64_t a = smem_desc(slots_addr + C::kRope * C::kSlotBytes + ks * 32, 16, 1024, 2);
             const uint64_t b = smem_desc(q_addr + C::NL * C::kQChunkBytes + ks * 32, 16, 1024, 2);
-            mma_bf16_ss(d_s, a, b, C::kIdescQK, ks > 0 ? 1u : 0u);
+            mma_bf16_ss(d_s + (ks % C::kChains) * NH, a, b, C::kIdescQK, ks >= C::kChains ? 1u : 0u);
           }
           mma_commit(&slot_empty[C::kRope]);
           for (int c = 0; c < C::NL && ok; ++c) {
@@ -346,7 +375,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t a = smem_desc(slots_addr + c * C::kSlotBytes + ks * 32, 16, 1024, 2);
               const uint64_t b = smem_desc(q_addr + c * C::kQChunkBytes + ks * 32, 16, 1024, 2);
-              mma_bf16_ss(d_s, a, b, C::kIdescQK, 1u);
+              const bool fresh = c == 0 && ks >= C::kRopeSteps;  // chain not yet written this tile
+              mma_bf16_ss(d_s + ks * NH, a, b, C::kIdescQK, fresh ? 0u : 1u);
             }
           }
           if (!ok) break;
@@ -357,21 +387,20 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           if (j == 0 && !(ok = mbar_wait(&o_empty[ob], ((qi >> 1) & 1) ^ 1, abort_flag, p.ws, 35)))
             break;
           tc_fence_after();
-#pragma unroll 1
-          for (int mb = 0; mb < C::MB; ++mb) {
-            const uint32_t d_o = tmem_base + C::kTmemO + (ob * C::MB + mb) * NH;
+          // the MB output blocks are independent accumulators: interleave them
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t b = smem_desc(p_addr + pb * C::kPBytes + kk * 16 * C::kPRowBytes,
+                                         8 * C::kPRowBytes, 8 * C::kPRowBytes, C::kPSwz);
+#pragma unroll
+            for (int mb = 0; mb < C::MB; ++mb) {
+              const uint32_t d_o = tmem_base + C::kTmemO + (ob * C::MB + mb) * NH;
               const uint64_t a = smem_desc(slots_addr + (2 * mb) * C::kSlotBytes + kk * 2048,
                                            C::kSlotBytes, 1024, 2);
-              const uint64_t b = smem_desc(p_addr + pb * C::kPBytes + (kk >> 2) * C::kQChunkBytes +
-                                               (kk & 3) * 32,
-                                           16, 1024, 2);
               mma_bf16_ss(d_o, a, b, C::kIdescPV, (j == 0 && kk == 0) ? 0u : 1u);
             }
-            if (2 * mb < C::NL) mma_commit(&slot_empty[2 * mb]);
-            if (2 * mb + 1 < C::NL) mma_commit(&slot_empty[2 * mb + 1]);
           }
+          for (int c = 0; c < C::NL; ++c) mma_commit(&slot_empty[c]);
           mma_commit(&p_empty[pb]);
           mma_commit(o_step);
           if (j == nt - 1) mma_commit(&o_full[ob]);
@@ -408,7 +437,14 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         float x[NH];
-        tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * NH, x);
+        tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * C::kChains * NH, x);
+#pragma unroll
+        for (int ch = 1; ch < C::kChains; ++ch) {
+          float y[NH];
+          tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + (sb * C::kChains + ch) * NH, y);
+#pragma unroll
+          for (int h = 0; h < NH; ++h) x[h] += y[h];
+        }
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
         const bool valid = row >= 0 && row < p.ctx_len;
@@ -460,16 +496,29 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         ok = __all_sync(0xffffffffu,
                         mbar_wait(&p_empty[pb], ((tc >> 1) & 1) ^ 1, abort_flag, p.ws, 43));
         if (!ok) break;
-        unsigned char* pt = sP + pb * C::kPBytes + (r >> 6) * C::kQChunkBytes;
-        const int e = r & 63;
+        // this key's row of P: NH bf16, written as 16-byte chunks at their
+        // swizzled positions (chunk c ^ ((r >> 1) & 3) for 64-byte rows,
+        // c ^ ((r >> 2) & 1) for 32-byte rows)
+        uint32_t packed[NH / 2];
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-          float pv = 0.f;
-          if (x[h] > -INFINITY && mrep[h] > -INFINITY) pv = ex2_approx(x[h] - mrep[h]);
-          const uint16_t b = f32_to_bf16_rne(pv);
-          lpart[h] += bf16_to_f32(b);
-          *reinterpret_cast<uint16_t*>(pt + h * 128 + (((e >> 3) ^ (h & 7)) << 4) + (e & 7) * 2) = b;
+        for (int h2 = 0; h2 < NH / 2; ++h2) {
+          float pv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = 2 * h2 + e;
+            pv[e] = 0.f;
+            if (h < H && x[h] > -INFINITY && mrep[h] > -INFINITY) pv[e] = ex2_approx(x[h] - mrep[h]);
+            lpart[h] += pv[e];
+          }
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
+          packed[h2] = *reinterpret_cast<const uint32_t*>(&b2);
         }
+        unsigned char* prow = sP + pb * C::kPBytes + r * C::kPRowBytes;
+        const int swz = NH == 32 ? ((r >> 1) & 3) : ((r >> 2) & 1);
+#pragma unroll
+        for (int c = 0; c < NH / 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) =
+              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&p_full[pb]);
@@ -546,12 +595,25 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
   p.prefix_valid = prefix_valid ? 1 : 0;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.ws = ws;
+  CUtensorMap tm_lat, tm_rope, tm_q;
+  if (!make_tmap_bf16_2d(&tm_lat, latent, DC, static_cast<uint64_t>(d.ctx_len), 64, 1,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_bf16_2d(&tm_q, q, DC + DR, static_cast<uint64_t>(d.n_q) * H, 64, H,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (C::kRopeTma) {
+    if (!make_tmap_bf16_2d(&tm_rope, rope, DR, static_cast<uint64_t>(d.ctx_len), 64, 1,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
+    tm_rope = tm_lat;  // unused
+  }
   const int grid = d.n_q < num_sms() ? d.n_q : num_sms();
   const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc<H, DC, DR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  sparse_attn_tc<H, DC, DR><<<grid, C::kThreads, smem, st>>>(p);
+  sparse_attn_tc<H, DC, DR><<<grid, C::kThreads, smem, st>>>(tm_lat, tm_rope, tm_q, p);
   return cudaGetLastError();
 }
 
