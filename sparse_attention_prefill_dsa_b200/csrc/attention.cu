@@ -14,32 +14,37 @@
 // share each gathered row.
 //
 // Per query, in tiles of 128 selected keys:
-//   gather   latent (8 x 64-dim chunks) and rope rows of the tile into nine
-//            16 KB shared-memory slots, 128-byte swizzled, one key per 128-byte
-//            row, with TMA tile::gather4 loads (four selected rows each);
+//   gather   the tile's rope chunk and its latent rows, as 128-dim pairs of
+//            64-dim chunks (one 32 KB pair per PV output block), into
+//            shared memory with cp.async: one key per 128-byte row, 128-byte
+//            swizzled, eight threads per row so every request is a full
+//            128-byte line. Pairs form a ring one pair deeper than a tile, so
+//            the next tile's rope and first pair arrive during the softmax;
 //   QK^T     S^T[key, head] = K_tile . Q^T: keys are the MMA's M (128), the
-//            padded heads its N, K = Dc + Dr, both operands K-major; rope
-//            chunk first so its slot is released earliest. A tcgen05.mma that
-//            depends on the previous one's accumulator waits out its latency,
-//            so the K steps feed four independent partial sums (summed by the
-//            softmax) and the PV interleaves its four 128-dim output blocks;
+//            padded heads its N, K = Dc + Dr, both operands K-major;
 //   softmax  one thread per key lane of S^T: the per-head tile maximum is found
 //            with a warp transpose-reduction plus a four-warp exchange through
 //            shared memory (mbarrier-synchronised), the running maximum is
-//            raised only when a tile exceeds it by more than 2^8 (then O and
-//            the partial sums are rescaled), and p = 2^(z log2e - m) is written
-//            as bf16 into P [key, head] (one 16-byte-chunked row per key);
-//   PV       O^T[dim, head] += latent_tile^T . P^T: the same latent slots read
-//            MN-major as A (dims as M, four 128-dim blocks), P MN-major as B;
-//            each block's two slots are released as soon as its MMAs finish,
-//            so the next tile's gather overlaps the current PV.
-// Accumulators live in TMEM (S^T double-buffered per tile, O^T per query);
-// the epilogue divides by the row sum, rounds to bf16 and writes out / lse.
+//            raised only when a tile exceeds it by more than 2^8 (then O is
+//            rescaled in TMEM), and p = 2^(z log2e - m) is written as bf16 into
+//            P [key, head] (one 16-byte-chunked row per key);
+//   PV       O^T[dim, head] += latent_tile^T . P^T: the latent pairs read
+//            MN-major as A (dims as M, one 128-dim block per pair), P MN-major
+//            as B. Each pair is released the moment its block's MMAs finish,
+//            so the next tile's gather runs under the current PV.
+// The MMA issuer orders its work as QK^T(t) on the rope and first pair,
+// PV(t-1), then QK^T(t) on the rest, so the tensor pipe works while the
+// gather of tile t completes. Accumulators live in TMEM (S^T double-buffered
+// per tile, O^T per query); the epilogue divides by the row sum, rounds to
+// bf16 and writes out / lse.
 //
 // Roles (288 threads, one CTA per SM, persistent over queries):
-//   warps 0-3  producers: cp.async gathers and the query's q rows;
-//   warp  4    TMEM owner and single-thread tcgen05.mma issuer;
-//   warps 5-8  softmax and epilogue (TMEM lanes 0-127 = keys, then dims).
+//   warps 0-3  producers: cp.async gathers of every tile;
+//   warp  4    TMEM owner and tcgen05.mma issuer (warp-collective, one
+//              elected lane issues);
+//   warps 5-8  softmax and epilogue (TMEM lanes 0-127 = keys, then dims); one
+//              lane also loads each query's q rows with 2D TMA once the
+//              previous query's last QK^T has completed.
 // Every wait is bounded; on a timeout the CTA records DSA_ERR_TIMEOUT, all
 // roles stop, copies and MMAs in flight are drained and TMEM is freed.
 #include <cuda_bf16.h>
@@ -60,12 +65,11 @@ struct AttnCfg {
   static constexpr int kKeys = 128;                   // keys per tile (MMA M of QK^T)
   static constexpr int NH = H < 16 ? 16 : H;          // heads padded to a legal MMA N
   static constexpr int NL = DC / 64;                  // latent 64-dim chunks
-  static constexpr int MB = (DC + 127) / 128;         // 128-dim blocks of the PV
-  static constexpr int NLS = 2 * MB;                  // latent slots (zero-padded)
-  static constexpr int kRope = NLS;                   // slot index of the rope chunk
-  static constexpr int kSlots = NLS + 1;
+  static constexpr int MB = (DC + 127) / 128;         // 128-dim PV blocks = latent pairs per tile
   static constexpr int kRopeSteps = DR / 16;
-  static constexpr int kSlotBytes = kKeys * 128;      // 16 KB
+  static constexpr int kChunkBytes = kKeys * 128;     // 16 KB: 64 dims of 128 keys
+  static constexpr int kPairBytes = 2 * kChunkBytes;  // one PV block (upper half zero if DC < 128)
+  static constexpr int kPairs = MB + 1 > 3 ? MB + 1 : 3;  // ring: one tile plus one pair
   static constexpr int kQChunks = NL + 1;             // latent chunks + rope chunk
   static constexpr int kQChunkBytes = NH * 128;
   // P: one row of NH bf16 per key (MN-major B operand of the PV), 64- or
@@ -73,31 +77,33 @@ struct AttnCfg {
   static constexpr int kPRowBytes = NH * 2;
   static constexpr int kPBytes = kKeys * kPRowBytes;
   static constexpr uint32_t kPSwz = NH == 32 ? 4u : 6u;  // descriptor code: 64B / 32B swizzle
+  static constexpr int kProducerThreads = 128;        // warps 0-3
   static constexpr int kThreads = 288;
-  static constexpr int kGatherPositions = NL + 1;     // rope, L0..L(NL-1)
-  static constexpr bool kRopeTma = DR == 64;          // a 128-byte rope row: TMA gather4
+  static constexpr int kRowsPerThread = kKeys / 16;   // keys 32w + lane/8 + 4i, i < 8
   static constexpr uint32_t kQBytes = H * 128 * kQChunks;  // q boxes (zero-filled past Dc+Dr)
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, NH, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, NH, true, true);
-  // TMEM columns: S^T[2 buffers][kChains partial sums] then O^T[2][MB]
-  static constexpr int kChains = 4;                   // independent QK^T accumulators
+  // TMEM columns: S^T[2] then O^T[2 queries][MB]
   static constexpr int kTmemS = 0;
-  static constexpr int kTmemO = 2 * kChains * NH;
-  static constexpr int kTmemUsed = 2 * kChains * NH + 2 * MB * NH;
+  static constexpr int kTmemO = 2 * NH;
+  static constexpr int kTmemUsed = 2 * NH + 2 * MB * NH;
   static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
   // shared memory carve (from a 1024-byte aligned base)
-  static constexpr int kOffSlots = 0;
-  static constexpr int kOffQ = kOffSlots + kSlots * kSlotBytes;
+  static constexpr int kOffPairs = 0;
+  static constexpr int kOffRope = kOffPairs + kPairs * kPairBytes;
+  static constexpr int kOffQ = kOffRope + kChunkBytes;
   static constexpr int kOffP = kOffQ + kQChunks * kQChunkBytes;
-  static constexpr int kOffRed = kOffP + 2 * kPBytes;            // [2][4][32] floats
+  static constexpr int kOffRed = kOffP + kPBytes;                // [2][4][32] floats
   static constexpr int kOffBar = kOffRed + 2 * 4 * 32 * 4;
-  static constexpr int kNumBars = 2 * kSlots + 2 + 2 * 2 + 2 * 2 + 2 * 2 + 1 + 2 + 1;
+  static constexpr int kNumBars = 3 * kPairs + 16;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(DC % 64 == 0 && DR % 16 == 0 && DR <= 64 && (NH % 16) == 0 && NH <= 32 &&
                     (H & (H - 1)) == 0,
                 "shape");
+  static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "operand alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct AttnParams {
@@ -113,9 +119,17 @@ struct AttnParams {
   WsHeader* ws;
 };
 
+__device__ __forceinline__ int n_valid_of(const AttnParams& p, int i) {
+  return p.prefix_valid ? min(p.k, p.q_pos0 + i + 1) : p.k;
+}
+
 __device__ __forceinline__ int n_tiles_of(const AttnParams& p, int i) {
-  const int valid = p.prefix_valid ? min(p.k, p.q_pos0 + i + 1) : p.k;
-  return (valid + 127) / 128;
+  return (n_valid_of(p, i) + 127) / 128;
+}
+
+// Selected key `sel` of query i, or -1 past the query's selection.
+__device__ __forceinline__ int selected_row(const AttnParams& p, int i, int sel) {
+  return sel < n_valid_of(p, i) ? __ldg(p.idx + static_cast<int64_t>(i) * p.k + sel) : -1;
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -183,29 +197,36 @@ __device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&x)[NH]
   }
 }
 
+// Shared-memory descriptor advanced by a byte offset (the start address is
+// the low field, in 16-byte units; every operand lies below 256 KB).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
+  return d + static_cast<uint64_t>(bytes >> 4);
+}
+
 template <int H, int DC, int DR>
 __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
-    sparse_attn_tc(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
-                   const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
+    sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
   using C = AttnCfg<H, DC, DR>;
   constexpr int NH = C::NH;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* sSlots = smem + C::kOffSlots;
+  unsigned char* sPairs = smem + C::kOffPairs;
+  unsigned char* sRope = smem + C::kOffRope;
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sP = smem + C::kOffP;
   float* sRed = reinterpret_cast<float*>(smem + C::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* slot_full = bars;                        // [kSlots]
-  uint64_t* slot_empty = bars + C::kSlots;           // [kSlots]
-  uint64_t* q_full = bars + 2 * C::kSlots;           // [1]
-  uint64_t* q_empty = q_full + 1;                    // [1]
-  uint64_t* s_full = q_empty + 1;                    // [2]
+  uint64_t* pair_full = bars;                        // [kPairs][2] (one per 64-dim chunk)
+  uint64_t* pair_empty = bars + 2 * C::kPairs;       // [kPairs]
+  uint64_t* rope_full = pair_empty + C::kPairs;      // [1]
+  uint64_t* rope_empty = rope_full + 1;              // [1]
+  uint64_t* q_full = rope_empty + 1;                 // [1]
+  uint64_t* s_full = q_full + 1;                     // [2]
   uint64_t* s_empty = s_full + 2;                    // [2]
-  uint64_t* p_full = s_empty + 2;                    // [2]
-  uint64_t* p_empty = p_full + 2;                    // [2]
-  uint64_t* o_full = p_empty + 2;                    // [2]
+  uint64_t* p_full = s_empty + 2;                    // [1]
+  uint64_t* p_empty = p_full + 1;                    // [1]
+  uint64_t* o_full = p_empty + 1;                    // [2]
   uint64_t* o_empty = o_full + 2;                    // [2]
   uint64_t* o_step = o_empty + 2;                    // [1]
   uint64_t* exch = o_step + 1;                       // [2]
@@ -215,29 +236,26 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // zero every operand buffer once: padded heads, padded latent slots and the
-  // unused part of a narrow rope chunk must read as zeros
+  // zero every operand buffer once: padded heads, the upper half of a pair
+  // when Dc < 128 and the unused part of a narrow rope chunk read as zeros
   for (int e = threadIdx.x * 16; e < C::kOffRed; e += C::kThreads * 16)
     *reinterpret_cast<uint4*>(smem + e) = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kSlots; ++s) {
-      // TMA slots complete on bytes after one arrive; a cp.async rope slot on
-      // the 32 noinc arrivals of its warp
-      mbar_init(&slot_full[s], (s == C::kRope && !C::kRopeTma) ? 32 : 1);
-      mbar_init(&slot_empty[s], 1);
-    }
+    for (int s = 0; s < 2 * C::kPairs; ++s) mbar_init(&pair_full[s], C::kProducerThreads);
+    for (int s = 0; s < C::kPairs; ++s) mbar_init(&pair_empty[s], 1);
+    mbar_init(rope_full, C::kProducerThreads);
+    mbar_init(rope_empty, 1);
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&s_empty[b], 128);
-      mbar_init(&p_full[b], 128);
-      mbar_init(&p_empty[b], 1);
       mbar_init(&o_full[b], 1);
       mbar_init(&o_empty[b], 128);
       mbar_init(&exch[b], 128);
     }
+    mbar_init(p_full, 128);
+    mbar_init(p_empty, 1);
     mbar_init(o_step, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -250,177 +268,191 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
 
   if (warp < 4) {
     // -------------------------------------------------------------- producers
-    // This warp fills gather positions w, w+4, ... of each tile (position 0 is
-    // the rope chunk, position 1+c latent chunk c). A slot of 128 keys is 32
-    // TMA gather4 loads, one per lane: lane l brings keys 4l..4l+3 (four
-    // 128-byte rows, 512 swizzled bytes) and the slot's mbarrier completes on
-    // its 16 KB of transactions. Warp 0 also loads the query's q rows with 2D
-    // TMA boxes. A 16-dim rope chunk (too narrow for a 128-byte swizzled box)
-    // is gathered with cp.async, each lane announcing its copies with
-    // cp.async.mbarrier.arrive.noinc.
-    if (warp == 0 && lane == 0) {
-      prefetch_tmap(&tm_lat);
-      prefetch_tmap(&tm_q);
-      if (C::kRopeTma) prefetch_tmap(&tm_rope);
-    }
-    uint32_t tc = 0, qi = 0;
-    bool ok = true;
-    int last_slot_parity = -1;  // parity of this warp's last issued slot fills (for draining)
-    int q_parity = -1;
-    for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
-      if (warp == 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (qi & 1) ^ 1, abort_flag, p.ws, 20));
-        if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, C::kQBytes);
-          for (int c = 0; c < C::kQChunks; ++c)
-            tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, i * H, q_full);
-        }
-        q_parity = qi & 1;
-      }
-      const int nt = n_tiles_of(p, i);
-      const int32_t* irow = p.idx + static_cast<int64_t>(i) * p.k;
-      for (int j = 0; j < nt && ok; ++j, ++tc) {
-        // rows of keys 4*lane .. 4*lane+3 (masked or out-of-range keys read row 0;
-        // their softmax weight is zero)
-        int r4[4];
+    // Thread (warp w, lane l) copies 16-byte part l%8 of keys 32w + l/8 + 4i
+    // (i < 8) of every chunk: each warp-wide cp.async moves four full
+    // 128-byte rows. A chunk's mbarrier completes on the noinc arrivals of all
+    // 128 producer threads. Row indices of the next tile are loaded while the
+    // current tile's copies are issued.
+    constexpr int R = C::kRowsPerThread;
+    const int kbase = 32 * warp + (lane >> 3);
+    const int part = lane & 7;
+    uint32_t doff[R];  // swizzled destination of each key's part in a chunk
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int sel = j * 128 + 4 * lane + e;
-          int row = sel < p.k ? __ldg(irow + sel) : -1;
+    for (int e = 0; e < R; ++e) {
+      const int key = kbase + 4 * e;
+      doff[e] = key * 128 + ((part ^ (key & 7)) << 4);
+    }
+    int cur[R], nxt[R];
+    if (blockIdx.x < p.n_q) {
+#pragma unroll
+      for (int e = 0; e < R; ++e) cur[e] = selected_row(p, blockIdx.x, kbase + 4 * e);
+    }
+    uint32_t tc = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x) {
+      const int nt = n_tiles_of(p, i);
+      for (int j = 0; j < nt && ok; ++j, ++tc) {
+        const int ni = j + 1 < nt ? i : i + gridDim.x;
+        const int nj = j + 1 < nt ? j + 1 : 0;
+        if (ni < p.n_q) {
+#pragma unroll
+          for (int e = 0; e < R; ++e) nxt[e] = selected_row(p, ni, nj * 128 + kbase + 4 * e);
+        }
+        const uint16_t* lsrc[R];
+        const uint16_t* rsrc[R];
+#pragma unroll
+        for (int e = 0; e < R; ++e) {
+          int row = cur[e];
           if (row >= p.ctx_len) {
             report(p.ws, kDevRange, static_cast<unsigned>(i));
             row = -1;
           }
-          r4[e] = row < 0 ? 0 : row;
+          if (row < 0) row = 0;  // masked key: any valid row, weight zero
+          lsrc[e] = p.latent + static_cast<int64_t>(row) * DC + part * 8;
+          rsrc[e] = p.rope + static_cast<int64_t>(row) * DR + part * 8;
         }
-        for (int pos = warp; pos < C::kGatherPositions; pos += 4) {
-          const int slot = pos == 0 ? C::kRope : pos - 1;
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(&slot_empty[slot], (tc & 1) ^ 1, abort_flag, p.ws, 21));
+        ok = __all_sync(0xffffffffu, mbar_wait(rope_empty, (tc & 1) ^ 1, abort_flag, p.ws, 20));
+        if (!ok) break;
+        if (part < DR / 8) {
+#pragma unroll
+          for (int e = 0; e < R; ++e) cp_async_16(sRope + doff[e], rsrc[e]);
+        }
+        cp_async_arrive_noinc(rope_full);
+#pragma unroll
+        for (int mb = 0; mb < C::MB; ++mb) {
+          const uint32_t seq = C::MB * tc + mb;
+          const uint32_t pi = seq % C::kPairs;
+          ok = __all_sync(0xffffffffu, mbar_wait(&pair_empty[pi], ((seq / C::kPairs) & 1) ^ 1,
+                                                 abort_flag, p.ws, 21));
           if (!ok) break;
-          unsigned char* dst = sSlots + slot * C::kSlotBytes;
-          if (slot != C::kRope || C::kRopeTma) {
-            if (lane == 0) mbar_arrive_expect_tx(&slot_full[slot], C::kSlotBytes);
-            __syncwarp();
-            if (slot == C::kRope)
-              tma_gather4(dst + lane * 512, &tm_rope, 0, r4[0], r4[1], r4[2], r4[3], &slot_full[slot]);
-            else
-              tma_gather4(dst + lane * 512, &tm_lat, slot * 64, r4[0], r4[1], r4[2], r4[3],
-                          &slot_full[slot]);
-          } else {
-            const int part = lane & 7;
-            if (part < DR / 8) {
-#pragma unroll 4
-              for (int it = 0; it < 32; ++it) {
-                const int key = (lane >> 3) + 4 * it;
-                const int sel = j * 128 + key;
-                int row = sel < p.k ? __ldg(irow + sel) : -1;
-                if (row < 0 || row >= p.ctx_len) row = 0;
-                cp_async_16(dst + key * 128 + ((part ^ (key & 7)) << 4),
-                            p.rope + static_cast<int64_t>(row) * DR + part * 8);
-              }
+          unsigned char* dst = sPairs + pi * C::kPairBytes;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int c = 2 * mb + half;
+            if (c < C::NL) {
+#pragma unroll
+              for (int e = 0; e < R; ++e)
+                cp_async_16(dst + half * C::kChunkBytes + doff[e], lsrc[e] + c * 64);
+              cp_async_arrive_noinc(&pair_full[2 * pi + half]);
             }
-            cp_async_arrive_noinc(&slot_full[slot]);
           }
-          last_slot_parity = tc & 1;
         }
+#pragma unroll
+        for (int e = 0; e < R; ++e) cur[e] = nxt[e];
       }
     }
-    cp_async_wait_all();  // every cp.async copy lands before the CTA can exit
-    if (!ok && lane == 0) {  // and every TMA load this warp issued
-      if (last_slot_parity >= 0)
-        for (int pos = warp; pos < C::kGatherPositions; pos += 4) {
-          const int slot = pos == 0 ? C::kRope : pos - 1;
-          if (slot != C::kRope || C::kRopeTma) drain_wait(&slot_full[slot], last_slot_parity);
-        }
-      if (q_parity >= 0) drain_wait(q_full, q_parity);
-    }
+    cp_async_wait_all();  // every copy lands before the CTA can exit
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t tc = 0, qi = 0;
-      bool ok = true;
-      const uint32_t slots_addr = smem_u32(sSlots);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
-      for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
-        const int nt = n_tiles_of(p, i);
-        const int ob = qi & 1;
-        if (!(ok = mbar_wait(q_full, qi & 1, abort_flag, p.ws, 30))) break;
+    const uint64_t dq = smem_desc(smem_u32(sQ), 16, 1024, 2);
+    const uint64_t drope = smem_desc(smem_u32(sRope), 16, 1024, 2);
+    const uint64_t dpair_k = smem_desc(smem_u32(sPairs), 16, 1024, 2);
+    const uint64_t dpair_mn = smem_desc(smem_u32(sPairs), C::kChunkBytes, 1024, 2);
+    const uint64_t dp = smem_desc(smem_u32(sP), 8 * C::kPRowBytes, 8 * C::kPRowBytes, C::kPSwz);
+    auto wait = [&](uint64_t* bar, uint32_t parity, unsigned site) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.ws, site));
+    };
+    // QK^T on latent pair mb of tile tc (both chunks as they land)
+    auto qk_pair = [&](uint32_t tc, int mb, uint32_t d_s) {
+      const uint32_t seq = C::MB * tc + mb;
+      const uint32_t pi = seq % C::kPairs;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int c = 2 * mb + half;
+        if (c >= C::NL) break;
+        if (!wait(&pair_full[2 * pi + half], (seq / C::kPairs) & 1, 33)) return false;
         fence_proxy_async_smem();
-        for (int j = 0; j < nt; ++j, ++tc) {
-          const int sb = tc & 1, pb = tc & 1;
-          // ---- S^T = K_tile . Q^T
-          if (!(ok = mbar_wait(&s_empty[sb], ((tc >> 1) & 1) ^ 1, abort_flag, p.ws, 31))) break;
-          // S^T accumulates in kChains independent partial sums (K-step ks of
-          // every chunk goes to chain ks), so consecutive MMAs never wait on
-          // each other's accumulator; the softmax adds the partials.
-          const uint32_t d_s = tmem_base + C::kTmemS + sb * C::kChains * NH;
-          if (!(ok = mbar_wait(&slot_full[C::kRope], tc & 1, abort_flag, p.ws, 32))) break;
-          fence_proxy_async_smem();
-          tc_fence_after();
+        tc_fence_after();
+        const uint64_t a = desc_add(dpair_k, pi * C::kPairBytes + half * C::kChunkBytes);
+        const uint64_t b = desc_add(dq, c * C::kQChunkBytes);
 #pragma unroll
-          for (int ks = 0; ks < C::kRopeSteps; ++ks) {
-            const uint64_t a = smem_desc(slots_addr + C::kRope * C::kSlotBytes + ks * 32, 16, 1024, 2);
-            const uint64_t b = smem_desc(q_addr + C::NL * C::kQChunkBytes + ks * 32, 16, 1024, 2);
-            mma_bf16_ss(d_s + (ks % C::kChains) * NH, a, b, C::kIdescQK, ks >= C::kChains ? 1u : 0u);
-          }
-          mma_commit(&slot_empty[C::kRope]);
-          for (int c = 0; c < C::NL && ok; ++c) {
-            if (!(ok = mbar_wait(&slot_full[c], tc & 1, abort_flag, p.ws, 33))) break;
-            fence_proxy_async_smem();
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t a = smem_desc(slots_addr + c * C::kSlotBytes + ks * 32, 16, 1024, 2);
-              const uint64_t b = smem_desc(q_addr + c * C::kQChunkBytes + ks * 32, 16, 1024, 2);
-              const bool fresh = c == 0 && ks >= C::kRopeSteps;  // chain not yet written this tile
-              mma_bf16_ss(d_s + ks * NH, a, b, C::kIdescQK, fresh ? 0u : 1u);
-            }
-          }
-          if (!ok) break;
-          mma_commit(&s_full[sb]);
-          if (j == nt - 1) mma_commit(q_empty);
-          // ---- O^T += latent_tile^T . P^T
-          if (!(ok = mbar_wait(&p_full[pb], (tc >> 1) & 1, abort_flag, p.ws, 34))) break;
-          if (j == 0 && !(ok = mbar_wait(&o_empty[ob], ((qi >> 1) & 1) ^ 1, abort_flag, p.ws, 35)))
-            break;
-          tc_fence_after();
-          // the MB output blocks are independent accumulators: interleave them
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t b = smem_desc(p_addr + pb * C::kPBytes + kk * 16 * C::kPRowBytes,
-                                         8 * C::kPRowBytes, 8 * C::kPRowBytes, C::kPSwz);
-#pragma unroll
-            for (int mb = 0; mb < C::MB; ++mb) {
-              const uint32_t d_o = tmem_base + C::kTmemO + (ob * C::MB + mb) * NH;
-              const uint64_t a = smem_desc(slots_addr + (2 * mb) * C::kSlotBytes + kk * 2048,
-                                           C::kSlotBytes, 1024, 2);
-              mma_bf16_ss(d_o, a, b, C::kIdescPV, (j == 0 && kk == 0) ? 0u : 1u);
-            }
-          }
-          for (int c = 0; c < C::NL; ++c) mma_commit(&slot_empty[c]);
-          mma_commit(&p_empty[pb]);
-          mma_commit(o_step);
-          if (j == nt - 1) mma_commit(&o_full[ob]);
-        }
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16_ss_warp(d_s, desc_add(a, ks * 32), desc_add(b, ks * 32), C::kIdescQK, 1u);
       }
-      mma_commit(mma_done);
-      drain_wait(mma_done, 0);
+      return true;
+    };
+    // the PV of a finished tile, releasing each pair as its block completes
+    bool pend = false, pend_first = false, pend_last = false;
+    uint32_t pend_tc = 0, pend_qi = 0;
+    auto pv = [&]() {
+      if (!wait(p_full, pend_tc & 1, 34)) return false;
+      if (pend_first && !wait(&o_empty[pend_qi & 1], ((pend_qi >> 1) & 1) ^ 1, 35)) return false;
+      tc_fence_after();
+      const uint32_t d_o = tmem_base + C::kTmemO + (pend_qi & 1) * C::MB * NH;
+#pragma unroll
+      for (int mb = 0; mb < C::MB; ++mb) {
+        const uint32_t pi = (C::MB * pend_tc + mb) % C::kPairs;
+        const uint64_t a = desc_add(dpair_mn, pi * C::kPairBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss_warp(d_o + mb * NH, desc_add(a, kk * 2048), desc_add(dp, kk * 16 * C::kPRowBytes),
+                           C::kIdescPV, (pend_first && kk == 0) ? 0u : 1u);
+        mma_commit_warp(&pair_empty[pi]);
+      }
+      mma_commit_warp(p_empty);
+      mma_commit_warp(o_step);
+      if (pend_last) mma_commit_warp(&o_full[pend_qi & 1]);
+      pend = false;
+      return true;
+    };
+    uint32_t tc = 0, qi = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
+      const int nt = n_tiles_of(p, i);
+      for (int j = 0; j < nt; ++j, ++tc) {
+        const int sb = tc & 1;
+        const uint32_t d_s = tmem_base + C::kTmemS + sb * NH;
+        if (j == 0) {
+          // a new query: the previous query's last PV goes first, then q
+          if (pend && !(ok = pv())) break;
+          if (!(ok = wait(q_full, qi & 1, 30))) break;
+          tc_fence_after();
+        }
+        if (!(ok = wait(&s_empty[sb], ((tc >> 1) & 1) ^ 1, 31))) break;
+        if (!(ok = wait(rope_full, tc & 1, 32))) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < C::kRopeSteps; ++ks)
+          mma_bf16_ss_warp(d_s, desc_add(drope, ks * 32), desc_add(dq, C::NL * C::kQChunkBytes + ks * 32),
+                           C::kIdescQK, ks > 0 ? 1u : 0u);
+        mma_commit_warp(rope_empty);
+        if (!(ok = qk_pair(tc, 0, d_s))) break;
+        if (pend && !(ok = pv())) break;
+        for (int mb = 1; mb < C::MB && ok; ++mb) ok = qk_pair(tc, mb, d_s);
+        if (!ok) break;
+        mma_commit_warp(&s_full[sb]);
+        pend = true;
+        pend_tc = tc;
+        pend_qi = qi;
+        pend_first = j == 0;
+        pend_last = j == nt - 1;
+      }
     }
+    if (ok && pend) ok = pv();
+    mma_commit_warp(mma_done);
+    drain_wait(mma_done, 0);
   } else {
     // ------------------------------------------------- softmax and epilogue
     const int quarter = warp & 3;               // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;          // key lane (and dim lane in the epilogue)
     const int sw = warp - 5;                    // softmax warp index 0..3
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool q_loader = warp == 5 && lane == 0;
+    int q_loads = 0;
+    if (q_loader && blockIdx.x < p.n_q) {
+      prefetch_tmap(&tm_q);
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      for (int c = 0; c < C::kQChunks; ++c)
+        tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, blockIdx.x * H, q_full);
+      q_loads = 1;
+    }
     uint32_t tc = 0, qi = 0, xc = 0;
     bool ok = true;
+    int row_next = blockIdx.x < p.n_q ? selected_row(p, blockIdx.x, r) : -1;
     for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
       const int nt = n_tiles_of(p, i);
       const int ob = qi & 1;
-      const int32_t* irow = p.idx + static_cast<int64_t>(i) * p.k;
       float m_lane = -INFINITY;       // running max (log2 units) of head `lane`
       float mrep[NH];                 // running max of every head, replicated
       float lpart[NH];                // this key lane's share of the row sums
@@ -430,23 +462,27 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         lpart[h] = 0.f;
       }
       for (int j = 0; j < nt; ++j, ++tc) {
-        const int sb = tc & 1, pb = tc & 1;
-        const int sel = j * 128 + r;
-        const int row = sel < p.k ? __ldg(irow + sel) : -1;  // issued before the wait
+        const int sb = tc & 1;
+        const int row = row_next;
+        {
+          const int ni = j + 1 < nt ? i : i + static_cast<int>(gridDim.x);
+          const int nj = j + 1 < nt ? j + 1 : 0;
+          row_next = ni < p.n_q ? selected_row(p, ni, nj * 128 + r) : -1;
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (tc >> 1) & 1, abort_flag, p.ws, 40));
         if (!ok) break;
         tc_fence_after();
         float x[NH];
-        tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * C::kChains * NH, x);
-#pragma unroll
-        for (int ch = 1; ch < C::kChains; ++ch) {
-          float y[NH];
-          tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + (sb * C::kChains + ch) * NH, y);
-#pragma unroll
-          for (int h = 0; h < NH; ++h) x[h] += y[h];
-        }
+        tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * NH, x);
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
+        if (j == nt - 1 && q_loader && i + static_cast<int>(gridDim.x) < p.n_q) {
+          // every QK^T of query i has completed: bring in the next query's q
+          mbar_arrive_expect_tx(q_full, C::kQBytes);
+          for (int c = 0; c < C::kQChunks; ++c)
+            tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, (i + gridDim.x) * H, q_full);
+          ++q_loads;
+        }
         const bool valid = row >= 0 && row < p.ctx_len;
 #pragma unroll
         for (int h = 0; h < NH; ++h) x[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;
@@ -492,9 +528,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             tmem_st_wait();
           }
         }
-        // probabilities of this key for every head, bf16, into P^T[pb][h][r]
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&p_empty[pb], ((tc >> 1) & 1) ^ 1, abort_flag, p.ws, 43));
+        // the previous tile's PV has finished reading P
+        ok = __all_sync(0xffffffffu, mbar_wait(p_empty, (tc & 1) ^ 1, abort_flag, p.ws, 43));
         if (!ok) break;
         // this key's row of P: NH bf16, written as 16-byte chunks at their
         // swizzled positions (chunk c ^ ((r >> 1) & 3) for 64-byte rows,
@@ -513,7 +548,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
           packed[h2] = *reinterpret_cast<const uint32_t*>(&b2);
         }
-        unsigned char* prow = sP + pb * C::kPBytes + r * C::kPRowBytes;
+        unsigned char* prow = sP + r * C::kPRowBytes;
         const int swz = NH == 32 ? ((r >> 1) & 3) : ((r >> 2) & 1);
 #pragma unroll
         for (int c = 0; c < NH / 8; ++c)
@@ -521,7 +556,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
               make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&p_full[pb]);
+        mbar_arrive(p_full);
       }
       if (!ok) break;
       // ---- epilogue of query i
@@ -558,6 +593,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       tc_fence_before();
       mbar_arrive(&o_empty[ob]);
     }
+    // a q load that nobody consumed lands before the CTA exits
+    if (!ok && q_loader && q_loads > 0) drain_wait(q_full, (q_loads - 1) & 1);
   }
 
   __syncthreads();
@@ -595,25 +632,16 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
   p.prefix_valid = prefix_valid ? 1 : 0;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.ws = ws;
-  CUtensorMap tm_lat, tm_rope, tm_q;
-  if (!make_tmap_bf16_2d(&tm_lat, latent, DC, static_cast<uint64_t>(d.ctx_len), 64, 1,
-                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_bf16_2d(&tm_q, q, DC + DR, static_cast<uint64_t>(d.n_q) * H, 64, H,
+  CUtensorMap tm_q;
+  if (!make_tmap_bf16_2d(&tm_q, q, DC + DR, static_cast<uint64_t>(d.n_q) * H, 64, H,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (C::kRopeTma) {
-    if (!make_tmap_bf16_2d(&tm_rope, rope, DR, static_cast<uint64_t>(d.ctx_len), 64, 1,
-                           CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  } else {
-    tm_rope = tm_lat;  // unused
-  }
   const int grid = d.n_q < num_sms() ? d.n_q : num_sms();
   const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc<H, DC, DR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  sparse_attn_tc<H, DC, DR><<<grid, C::kThreads, smem, st>>>(tm_lat, tm_rope, tm_q, p);
+  sparse_attn_tc<H, DC, DR><<<grid, C::kThreads, smem, st>>>(tm_q, p);
   return cudaGetLastError();
 }
 
