@@ -22,12 +22,20 @@
 //            the next tile's rope and first pair arrive during the softmax;
 //   QK^T     S^T[key, head] = K_tile . Q^T: keys are the MMA's M (128), the
 //            padded heads its N, K = Dc + Dr, both operands K-major;
-//   softmax  one thread per key lane of S^T: the per-head tile maximum is found
-//            with a warp transpose-reduction plus a four-warp exchange through
-//            shared memory (mbarrier-synchronised), the running maximum is
-//            raised only when a tile exceeds it by more than 2^8 (then O is
-//            rescaled in TMEM), and p = 2^(z log2e - m) is written as bf16 into
-//            P [key, head] (one 16-byte-chunked row per key);
+//   softmax  one thread per key lane of S^T, p = 2^(z log2e - m) written as
+//            bf16 into P [key, head] (one 16-byte-chunked row per key). The
+//            reference m is a running maximum. On a query's first tile it is
+//            the tile maximum (a warp transpose-reduction plus a four-warp
+//            exchange through shared memory, mbarrier-synchronised). Every
+//            score of head h is at most B_h = |scale| log2e ||q_h|| max_s ||k_s||
+//            (Cauchy-Schwarz), so while B_h <= m_h + 64 for every head, p stays
+//            below 2^64 and no later tile can overflow fp32 or bf16: such
+//            tiles keep m as it is and skip the reduction and the exchange.
+//            Otherwise a tile takes the exact path, and m is raised only when
+//            the tile maximum exceeds it by more than 2^8 (then O is rescaled
+//            in TMEM). max_s ||k_s|| comes from a small pass over the keys
+//            before the attention kernel, ||q_h|| from the q rows in shared
+//            memory on the first tile;
 //   PV       O^T[dim, head] += latent_tile^T . P^T: the latent pairs read
 //            MN-major as A (dims as M, one 128-dim block per pair), P MN-major
 //            as B. Each pair is released the moment its block's MMAs finish,
@@ -95,8 +103,10 @@ struct AttnCfg {
   static constexpr int kOffQ = kOffRope + kChunkBytes;
   static constexpr int kOffP = kOffQ + kQChunks * kQChunkBytes;
   static constexpr int kOffRed = kOffP + kPBytes;                // [2][4][32] floats
-  static constexpr int kOffBar = kOffRed + 2 * 4 * 32 * 4;
-  static constexpr int kNumBars = 3 * kPairs + 16;
+  static constexpr int kOffNorm = kOffRed + 2 * 4 * 32 * 4;      // [4][32] floats
+  static constexpr int kOffM = kOffNorm + 4 * 32 * 4;            // [4 warps][32] floats
+  static constexpr int kOffBar = kOffM + 4 * 32 * 4;
+  static constexpr int kNumBars = 3 * kPairs + 17;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(DC % 64 == 0 && DR % 16 == 0 && DR <= 64 && (NH % 16) == 0 && NH <= 32 &&
@@ -203,6 +213,88 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
   return d + static_cast<uint64_t>(bytes >> 4);
 }
 
+// mbarrier layout (all in shared memory, after the operand buffers)
+template <class C>
+struct AttnBars {
+  static constexpr int kPairFull = 0;                  // [kPairs][2] (one per 64-dim chunk)
+  static constexpr int kPairEmpty = 2 * C::kPairs;     // [kPairs]
+  static constexpr int kRopeFull = 3 * C::kPairs;
+  static constexpr int kRopeEmpty = kRopeFull + 1;
+  static constexpr int kQFull = kRopeEmpty + 1;
+  static constexpr int kSFull = kQFull + 1;            // [2]
+  static constexpr int kSEmpty = kSFull + 2;           // [2]
+  static constexpr int kPFull = kSEmpty + 2;
+  static constexpr int kPEmpty = kPFull + 1;
+  static constexpr int kOFull = kPEmpty + 1;           // [2]
+  static constexpr int kOEmpty = kOFull + 2;           // [2]
+  static constexpr int kOStep = kOEmpty + 2;
+  static constexpr int kExch = kOStep + 1;             // [2]
+  static constexpr int kMmaDone = kExch + 2;
+  static constexpr int kCount = kMmaDone + 1;
+  static_assert(kCount == C::kNumBars, "barrier count");
+};
+
+// A wait by every lane of a warp, with one verdict for the whole warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          WsHeader* ws, unsigned site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, ws, site));
+}
+
+// QK^T on latent pair mb of tile tc, each chunk as soon as it lands
+// (warp-collective).
+template <class C>
+__device__ __forceinline__ bool attn_qk_pair(const AttnParams& p, volatile int* abort_flag, uint64_t* bars,
+                                             uint64_t dpair_k, uint64_t dq, uint32_t tc, int mb,
+                                             uint32_t d_s) {
+  using B = AttnBars<C>;
+  const uint32_t seq = C::MB * tc + mb;
+  const uint32_t pi = seq % C::kPairs;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int c = 2 * mb + half;
+    if (c >= C::NL) break;
+    if (!warp_wait(&bars[B::kPairFull + 2 * pi + half], (seq / C::kPairs) & 1, abort_flag, p.ws, 33))
+      return false;
+    fence_proxy_async_smem();
+    tc_fence_after();
+    const uint64_t a = desc_add(dpair_k, pi * C::kPairBytes + half * C::kChunkBytes);
+    const uint64_t b = desc_add(dq, c * C::kQChunkBytes);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+      mma_bf16_ss_warp(d_s, desc_add(a, ks * 32), desc_add(b, ks * 32), C::kIdescQK, 1u);
+  }
+  return true;
+}
+
+// O^T += latent_tile^T . P^T for tile tc of the qi-th query of this CTA,
+// releasing each latent pair as its block's MMAs complete (warp-collective).
+template <class C>
+__device__ __forceinline__ bool attn_pv(const AttnParams& p, volatile int* abort_flag, uint64_t* bars,
+                                        uint32_t tmem_base, uint64_t dpair_mn, uint64_t dp, uint32_t tc,
+                                        uint32_t qi, bool first, bool last) {
+  using B = AttnBars<C>;
+  constexpr int NH = C::NH;
+  if (!warp_wait(&bars[B::kPFull], tc & 1, abort_flag, p.ws, 34)) return false;
+  if (first && !warp_wait(&bars[B::kOEmpty + (qi & 1)], ((qi >> 1) & 1) ^ 1, abort_flag, p.ws, 35))
+    return false;
+  tc_fence_after();
+  const uint32_t d_o = tmem_base + C::kTmemO + (qi & 1) * C::MB * NH;
+#pragma unroll
+  for (int mb = 0; mb < C::MB; ++mb) {
+    const uint32_t pi = (C::MB * tc + mb) % C::kPairs;
+    const uint64_t a = desc_add(dpair_mn, pi * C::kPairBytes);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16_ss_warp(d_o + mb * NH, desc_add(a, kk * 2048), desc_add(dp, kk * 16 * C::kPRowBytes),
+                       C::kIdescPV, (first && kk == 0) ? 0u : 1u);
+    mma_commit_warp(&bars[B::kPairEmpty + pi]);
+  }
+  mma_commit_warp(&bars[B::kPEmpty]);
+  mma_commit_warp(&bars[B::kOStep]);
+  if (last) mma_commit_warp(&bars[B::kOFull + (qi & 1)]);
+  return true;
+}
+
 template <int H, int DC, int DR>
 __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     sparse_attn_tc(const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
@@ -216,21 +308,24 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sP = smem + C::kOffP;
   float* sRed = reinterpret_cast<float*>(smem + C::kOffRed);
+  float* sNorm = reinterpret_cast<float*>(smem + C::kOffNorm);
+  float* sM = reinterpret_cast<float*>(smem + C::kOffM);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* pair_full = bars;                        // [kPairs][2] (one per 64-dim chunk)
-  uint64_t* pair_empty = bars + 2 * C::kPairs;       // [kPairs]
-  uint64_t* rope_full = pair_empty + C::kPairs;      // [1]
-  uint64_t* rope_empty = rope_full + 1;              // [1]
-  uint64_t* q_full = rope_empty + 1;                 // [1]
-  uint64_t* s_full = q_full + 1;                     // [2]
-  uint64_t* s_empty = s_full + 2;                    // [2]
-  uint64_t* p_full = s_empty + 2;                    // [1]
-  uint64_t* p_empty = p_full + 1;                    // [1]
-  uint64_t* o_full = p_empty + 1;                    // [2]
-  uint64_t* o_empty = o_full + 2;                    // [2]
-  uint64_t* o_step = o_empty + 2;                    // [1]
-  uint64_t* exch = o_step + 1;                       // [2]
-  uint64_t* mma_done = exch + 2;                     // [1]
+  using B = AttnBars<C>;
+  uint64_t* pair_full = bars + B::kPairFull;
+  uint64_t* pair_empty = bars + B::kPairEmpty;
+  uint64_t* rope_full = bars + B::kRopeFull;
+  uint64_t* rope_empty = bars + B::kRopeEmpty;
+  uint64_t* q_full = bars + B::kQFull;
+  uint64_t* s_full = bars + B::kSFull;
+  uint64_t* s_empty = bars + B::kSEmpty;
+  uint64_t* p_full = bars + B::kPFull;
+  uint64_t* p_empty = bars + B::kPEmpty;
+  uint64_t* o_full = bars + B::kOFull;
+  uint64_t* o_empty = bars + B::kOEmpty;
+  uint64_t* o_step = bars + B::kOStep;
+  uint64_t* exch = bars + B::kExch;
+  uint64_t* mma_done = bars + B::kMmaDone;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -349,52 +444,10 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     const uint64_t dpair_k = smem_desc(smem_u32(sPairs), 16, 1024, 2);
     const uint64_t dpair_mn = smem_desc(smem_u32(sPairs), C::kChunkBytes, 1024, 2);
     const uint64_t dp = smem_desc(smem_u32(sP), 8 * C::kPRowBytes, 8 * C::kPRowBytes, C::kPSwz);
-    auto wait = [&](uint64_t* bar, uint32_t parity, unsigned site) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.ws, site));
-    };
-    // QK^T on latent pair mb of tile tc (both chunks as they land)
-    auto qk_pair = [&](uint32_t tc, int mb, uint32_t d_s) {
-      const uint32_t seq = C::MB * tc + mb;
-      const uint32_t pi = seq % C::kPairs;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int c = 2 * mb + half;
-        if (c >= C::NL) break;
-        if (!wait(&pair_full[2 * pi + half], (seq / C::kPairs) & 1, 33)) return false;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint64_t a = desc_add(dpair_k, pi * C::kPairBytes + half * C::kChunkBytes);
-        const uint64_t b = desc_add(dq, c * C::kQChunkBytes);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16_ss_warp(d_s, desc_add(a, ks * 32), desc_add(b, ks * 32), C::kIdescQK, 1u);
-      }
-      return true;
-    };
-    // the PV of a finished tile, releasing each pair as its block completes
+    // the PV of a finished tile (pend_*), issued once the next tile's first
+    // chunks are in
     bool pend = false, pend_first = false, pend_last = false;
     uint32_t pend_tc = 0, pend_qi = 0;
-    auto pv = [&]() {
-      if (!wait(p_full, pend_tc & 1, 34)) return false;
-      if (pend_first && !wait(&o_empty[pend_qi & 1], ((pend_qi >> 1) & 1) ^ 1, 35)) return false;
-      tc_fence_after();
-      const uint32_t d_o = tmem_base + C::kTmemO + (pend_qi & 1) * C::MB * NH;
-#pragma unroll
-      for (int mb = 0; mb < C::MB; ++mb) {
-        const uint32_t pi = (C::MB * pend_tc + mb) % C::kPairs;
-        const uint64_t a = desc_add(dpair_mn, pi * C::kPairBytes);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss_warp(d_o + mb * NH, desc_add(a, kk * 2048), desc_add(dp, kk * 16 * C::kPRowBytes),
-                           C::kIdescPV, (pend_first && kk == 0) ? 0u : 1u);
-        mma_commit_warp(&pair_empty[pi]);
-      }
-      mma_commit_warp(p_empty);
-      mma_commit_warp(o_step);
-      if (pend_last) mma_commit_warp(&o_full[pend_qi & 1]);
-      pend = false;
-      return true;
-    };
     uint32_t tc = 0, qi = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
@@ -404,12 +457,15 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         const uint32_t d_s = tmem_base + C::kTmemS + sb * NH;
         if (j == 0) {
           // a new query: the previous query's last PV goes first, then q
-          if (pend && !(ok = pv())) break;
-          if (!(ok = wait(q_full, qi & 1, 30))) break;
+          if (pend && !(ok = attn_pv<C>(p, abort_flag, bars, tmem_base, dpair_mn, dp, pend_tc, pend_qi,
+                                        pend_first, pend_last)))
+            break;
+          pend = false;
+          if (!(ok = warp_wait(q_full, qi & 1, abort_flag, p.ws, 30))) break;
           tc_fence_after();
         }
-        if (!(ok = wait(&s_empty[sb], ((tc >> 1) & 1) ^ 1, 31))) break;
-        if (!(ok = wait(rope_full, tc & 1, 32))) break;
+        if (!(ok = warp_wait(&s_empty[sb], ((tc >> 1) & 1) ^ 1, abort_flag, p.ws, 31))) break;
+        if (!(ok = warp_wait(rope_full, tc & 1, abort_flag, p.ws, 32))) break;
         fence_proxy_async_smem();
         tc_fence_after();
 #pragma unroll
@@ -417,9 +473,13 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           mma_bf16_ss_warp(d_s, desc_add(drope, ks * 32), desc_add(dq, C::NL * C::kQChunkBytes + ks * 32),
                            C::kIdescQK, ks > 0 ? 1u : 0u);
         mma_commit_warp(rope_empty);
-        if (!(ok = qk_pair(tc, 0, d_s))) break;
-        if (pend && !(ok = pv())) break;
-        for (int mb = 1; mb < C::MB && ok; ++mb) ok = qk_pair(tc, mb, d_s);
+        if (!(ok = attn_qk_pair<C>(p, abort_flag, bars, dpair_k, dq, tc, 0, d_s))) break;
+        if (pend && !(ok = attn_pv<C>(p, abort_flag, bars, tmem_base, dpair_mn, dp, pend_tc, pend_qi,
+                                      pend_first, pend_last)))
+          break;
+        pend = false;
+        for (int mb = 1; mb < C::MB && ok; ++mb)
+          ok = attn_qk_pair<C>(p, abort_flag, bars, dpair_k, dq, tc, mb, d_s);
         if (!ok) break;
         mma_commit_warp(&s_full[sb]);
         pend = true;
@@ -429,7 +489,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         pend_last = j == nt - 1;
       }
     }
-    if (ok && pend) ok = pv();
+    if (ok && pend)
+      ok = attn_pv<C>(p, abort_flag, bars, tmem_base, dpair_mn, dp, pend_tc, pend_qi, pend_first, pend_last);
     mma_commit_warp(mma_done);
     drain_wait(mma_done, 0);
   } else {
@@ -450,17 +511,22 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     uint32_t tc = 0, qi = 0, xc = 0;
     bool ok = true;
     int row_next = blockIdx.x < p.n_q ? selected_row(p, blockIdx.x, r) : -1;
+    // max_s ||k_s|| of the context, with the rounding slack of its float32 sum
+    const float kmax = __uint_as_float(*reinterpret_cast<volatile unsigned int*>(&p.ws->akmax_bits));
+    const float bound_scale = fabsf(p.scale_log2) * kmax;
     for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
       const int nt = n_tiles_of(p, i);
       const int ob = qi & 1;
+      const bool next_q = i + static_cast<int>(gridDim.x) < p.n_q;
       float m_lane = -INFINITY;       // running max (log2 units) of head `lane`
-      float mrep[NH];                 // running max of every head, replicated
+      float bound_lane = INFINITY;    // B_lane: bound on every score of head `lane`
+      bool fixed_m = false;           // B_h <= m_h + 64 for every head: keep m as it is
+      float* mrep = sM + sw * 32;     // running max of every head (this warp's copy)
       float lpart[NH];                // this key lane's share of the row sums
+      mrep[lane] = -INFINITY;
+      __syncwarp();
 #pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        mrep[h] = -INFINITY;
-        lpart[h] = 0.f;
-      }
+      for (int h = 0; h < NH; ++h) lpart[h] = 0.f;
       for (int j = 0; j < nt; ++j, ++tc) {
         const int sb = tc & 1;
         const int row = row_next;
@@ -476,57 +542,92 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * NH, x);
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
-        if (j == nt - 1 && q_loader && i + static_cast<int>(gridDim.x) < p.n_q) {
-          // every QK^T of query i has completed: bring in the next query's q
+        if (j == 0) {
+          // this warp's share of ||q_h||^2 (q chunks sw, sw+4, ...; lane = head),
+          // reading the 16-byte units of a row in a lane-rotated order
+          ok = __all_sync(0xffffffffu, mbar_wait(q_full, qi & 1, abort_flag, p.ws, 46));
+          if (!ok) break;
+          float qn2 = 0.f;
+          if (lane < NH) {
+            for (int c = sw; c < C::kQChunks; c += 4) {
+              const unsigned char* qrow = sQ + c * C::kQChunkBytes + lane * 128;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const uint4 v = *reinterpret_cast<const uint4*>(qrow + (((u + lane) & 7) << 4));
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float a = __uint_as_float(w[e] << 16), b = __uint_as_float(w[e] & 0xFFFF0000u);
+                  qn2 = fmaf(a, a, fmaf(b, b, qn2));
+                }
+              }
+            }
+            sNorm[sw * 32 + lane] = qn2;
+          }
+        }
+        const bool issue_q = j == nt - 1 && q_loader && next_q;
+        const bool valid = row >= 0 && row < p.ctx_len;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) x[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;
+        if (!fixed_m) {
+          // per-head maximum of this tile over all 128 keys
+          float red[NH];
+#pragma unroll
+          for (int h = 0; h < NH; ++h) red[h] = x[h];
+          const float wmax = warp_transpose_reduce<NH, true>(red);
+          float* xbuf = sRed + (xc & 1) * 128;
+          if (lane < NH) xbuf[sw * 32 + lane] = wmax;
+          mbar_arrive(&exch[xc & 1]);
+          ok = __all_sync(0xffffffffu, mbar_wait(&exch[xc & 1], (xc >> 1) & 1, abort_flag, p.ws, 41));
+          ++xc;
+          if (!ok) break;
+          float tmax = -INFINITY;
+          if (lane < NH)
+            tmax = fmaxf(fmaxf(xbuf[lane], xbuf[32 + lane]), fmaxf(xbuf[64 + lane], xbuf[96 + lane]));
+          if (j == 0 && lane < NH) {
+            const float qn2 = sNorm[lane] + sNorm[32 + lane] + sNorm[64 + lane] + sNorm[96 + lane];
+            // the float32 sums are within 2^-8 of exact; the slack covers them
+            bound_lane = bound_scale * sqrtf(qn2) * (1.f + 0.00390625f);
+          }
+          const bool need = lane < H && tmax > -INFINITY && (m_lane == -INFINITY || tmax > m_lane + 8.f);
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = fmaxf(m_lane, tmax);
+            const float alpha_lane = m_lane == -INFINITY ? 0.f : ex2_approx(m_lane - m_new);
+            m_lane = m_new;
+            float alpha[NH];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+              alpha[h] = __shfl_sync(0xffffffffu, alpha_lane, h);
+              lpart[h] *= alpha[h];
+            }
+            mrep[lane] = m_lane;
+            __syncwarp();
+            if (j > 0) {  // rescale O^T once the previous tile's PV is complete
+              ok = __all_sync(0xffffffffu, mbar_wait(o_step, (tc - 1) & 1, abort_flag, p.ws, 42));
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll 1
+              for (int mb = 0; mb < C::MB; ++mb) {
+                const uint32_t ta = tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH;
+                float o[NH];
+                tmem_ld_row<NH>(ta, o);
+#pragma unroll
+                for (int h = 0; h < NH; ++h) o[h] *= alpha[h];
+                tmem_st_row<NH>(ta, o);
+              }
+              tmem_st_wait();
+            }
+          }
+          // B_h <= m_h + 64 for every head: 2^(z - m) < 2^64 on every later tile
+          fixed_m = __all_sync(0xffffffffu, lane >= H || bound_lane <= m_lane + 64.f);
+        }
+        if (issue_q) {
+          // every QK^T of query i has completed and every warp has read its q
+          // rows (the first tile's exchange): bring in the next query's q
           mbar_arrive_expect_tx(q_full, C::kQBytes);
           for (int c = 0; c < C::kQChunks; ++c)
             tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, (i + gridDim.x) * H, q_full);
           ++q_loads;
-        }
-        const bool valid = row >= 0 && row < p.ctx_len;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) x[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;
-        // per-head maximum of this tile over all 128 keys
-        float red[NH];
-#pragma unroll
-        for (int h = 0; h < NH; ++h) red[h] = x[h];
-        const float wmax = warp_transpose_reduce<NH, true>(red);
-        float* xbuf = sRed + (xc & 1) * 128;
-        if (lane < NH) xbuf[sw * 32 + lane] = wmax;
-        mbar_arrive(&exch[xc & 1]);
-        ok = __all_sync(0xffffffffu, mbar_wait(&exch[xc & 1], (xc >> 1) & 1, abort_flag, p.ws, 41));
-        ++xc;
-        if (!ok) break;
-        float tmax = -INFINITY;
-        if (lane < NH)
-          tmax = fmaxf(fmaxf(xbuf[lane], xbuf[32 + lane]), fmaxf(xbuf[64 + lane], xbuf[96 + lane]));
-        const bool need = lane < H && tmax > -INFINITY && (m_lane == -INFINITY || tmax > m_lane + 8.f);
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = fmaxf(m_lane, tmax);
-          const float alpha_lane = m_lane == -INFINITY ? 0.f : ex2_approx(m_lane - m_new);
-          m_lane = m_new;
-          float alpha[NH];
-#pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            alpha[h] = __shfl_sync(0xffffffffu, alpha_lane, h);
-            mrep[h] = __shfl_sync(0xffffffffu, m_lane, h);
-            lpart[h] *= alpha[h];
-          }
-          if (j > 0) {  // rescale O^T once the previous tile's PV is complete
-            ok = __all_sync(0xffffffffu, mbar_wait(o_step, (tc - 1) & 1, abort_flag, p.ws, 42));
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int mb = 0; mb < C::MB; ++mb) {
-              const uint32_t ta = tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH;
-              float o[NH];
-              tmem_ld_row<NH>(ta, o);
-#pragma unroll
-              for (int h = 0; h < NH; ++h) o[h] *= alpha[h];
-              tmem_st_row<NH>(ta, o);
-            }
-            tmem_st_wait();
-          }
         }
         // the previous tile's PV has finished reading P
         ok = __all_sync(0xffffffffu, mbar_wait(p_empty, (tc & 1) ^ 1, abort_flag, p.ws, 43));
@@ -542,7 +643,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           for (int e = 0; e < 2; ++e) {
             const int h = 2 * h2 + e;
             pv[e] = 0.f;
-            if (h < H && x[h] > -INFINITY && mrep[h] > -INFINITY) pv[e] = ex2_approx(x[h] - mrep[h]);
+            const float mh = mrep[h];
+            if (h < H && x[h] > -INFINITY && mh > -INFINITY) pv[e] = ex2_approx(x[h] - mh);
             lpart[h] += pv[e];
           }
           const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
@@ -604,6 +706,37 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
   }
 }
 
+// max_s ||[latent_s, rope_s]||_2 over the context, one warp per key, as a
+// float32 bit pattern in the workspace header (non-negative floats order like
+// their bit patterns). Scaled up by 2^-8 to cover the float32 sums.
+template <int DC, int DR>
+__global__ void attn_key_norm_max_kernel(const uint16_t* __restrict__ latent,
+                                         const uint16_t* __restrict__ rope, int T, WsHeader* ws) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  float best = 0.f;
+  for (int s = warp; s < T; s += nwarps) {
+    float ss = 0.f;
+    const uint4* lr = reinterpret_cast<const uint4*>(latent + static_cast<int64_t>(s) * DC);
+    const uint4* rr = reinterpret_cast<const uint4*>(rope + static_cast<int64_t>(s) * DR);
+    for (int v = lane; v < (DC + DR) / 8; v += 32) {
+      const uint4 u = v < DC / 8 ? __ldg(lr + v) : __ldg(rr + (v - DC / 8));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = __uint_as_float(w[e] << 16), b = __uint_as_float(w[e] & 0xFFFF0000u);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    best = fmaxf(best, ss);
+  }
+  if (lane == 0 && best > 0.f)
+    atomicMax(&ws->akmax_bits, __float_as_uint(sqrtf(best) * (1.f + 0.00390625f)));
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -636,6 +769,12 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
   if (!make_tmap_bf16_2d(&tm_q, q, DC + DR, static_cast<uint64_t>(d.n_q) * H, 64, H,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  {
+    const int threads = 256;
+    int blocks = (d.ctx_len * 32 + threads - 1) / threads;
+    if (blocks > num_sms() * 8) blocks = num_sms() * 8;
+    attn_key_norm_max_kernel<DC, DR><<<blocks, threads, 0, st>>>(latent, rope, d.ctx_len, ws);
+  }
   const int grid = d.n_q < num_sms() ? d.n_q : num_sms();
   const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc<H, DC, DR>,
