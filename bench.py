@@ -38,7 +38,15 @@ import workloads  # noqa: E402
 SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_LAYER = 4  # indexer scores, key-norm max, top-k, sparse attention
+# DRAM bytes (read + write) per query of one kernel launch, from the ncu capture
+# named beside each entry; traffic scales with the query count (q rows, outputs,
+# index rows), so a launch's traffic is this figure times n_q. An entry is
+# removed whenever its kernel changes after the capture.
+PROFILED_DRAM_BYTES_PER_QUERY = {
+    "sparse_attn": (140.56e6 / 2048, "profiles/sparse_attn_tc_chunk2k_ctx8k.md"),
+}
+
+KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
 
 
 def load_peaks():
@@ -84,63 +92,95 @@ def barrier(world: int):
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while running."""
+    """Samples SM clocks and clock-event (throttle) reasons while running.
 
+    Reads NVML every few milliseconds from a background thread (read-only
+    queries); falls back to `nvidia-smi -lms` when NVML is unavailable.
+    """
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.005):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+        self.period = period_s
+        self.samples = []  # (sm_mhz, max_mhz, set of reason names)
+        self.stop = threading.Event()
         self.thread = None
+        self.proc = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            masks = [(n, getattr(pynvml, attr, 0)) for n, attr in self.REASONS]
+
+            def loop():
+                while not self.stop.is_set():
+                    try:
+                        mhz = pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM)
+                        bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                        self.samples.append((float(mhz), float(max_mhz),
+                                             {n for n, m in masks if m and bits & m}))
+                    except pynvml.NVMLError:
+                        pass
+                    self.stop.wait(self.period)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
             self.thread.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        except Exception:  # no NVML: sample with nvidia-smi instead
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "100", "-i", str(self.gpu)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._read_smi, daemon=True)
+                self.thread.start()
+            except (OSError, FileNotFoundError):
+                self.proc = None
         return self
 
-    def _read(self):
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                self.samples.append((float(parts[1]), float(parts[2]),
+                                     {n for n, v in zip(names, parts[5:9])
+                                      if v.lower().startswith("active")}))
+            except ValueError:
+                continue
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self.thread:
-                self.thread.join(timeout=2)
+        if self.thread:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": self.samples[-1][1], "reasons": sorted(reasons),
+                "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------ our GPU path
@@ -271,9 +311,12 @@ def run_ours(args):
     dom_flops = {"index_scores": fl["indexer"], "sparse_attn": fl["attention"]}
     if dom_name in dom_flops:
         ach = dom_flops[dom_name] / (per_kernel[dom_name] / 1e3) / 1e12
+        prof = PROFILED_DRAM_BYTES_PER_QUERY.get(dom_name)
         roof = {"kernel": dom_name, "bound": "tensor", "achieved": ach,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "frac": ach / peaks["bf16_tflops"],
+                "traffic": prof[0] * d.n_q if prof else None,
+                "traffic_source": (f"{prof[1]} (DRAM bytes per query x n_q)" if prof else None),
                 "peak_source": f"{peaks_src} bf16 burst (kernel timed alone)"}
     else:  # top-k reads the score rows once
         t = d.q_pos0 + np.arange(d.n_q)

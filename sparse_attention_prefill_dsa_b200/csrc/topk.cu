@@ -56,6 +56,15 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCandCap = 1024;
 constexpr int kMaxRounds = 48;
+// refine scratch: extra room that makes hist + cand + extra the float64 key
+// staging of the re-score (two keys of 128 dims per warp); the query's indexer
+// row (at most 32 x 128 bf16) in rows padded to an odd number of 32-bit words,
+// so that lane j reading row j hits bank (65 j + w) mod 32; the radix histogram
+// of the slow path
+constexpr int kKstExtraBytes = kWarps * 2 * 128 * 8 - kBins * 4 - kCandCap * 4;
+constexpr int kQRowBytes = 32 * (128 + 2) * 2;
+constexpr int kHist256Bytes = 256 * 4;
+static_assert(kKstExtraBytes >= 0 && kKstExtraBytes % 16 == 0, "key staging");
 
 constexpr double kDotRel = 1.0 / 32768.0;                  // 2^-15
 constexpr double kBoundRel = kDotRel + 1.0 / 131072.0;      // + 2^-17
@@ -73,6 +82,13 @@ struct Scratch {
 };
 
 __device__ __forceinline__ float canon(float f) { return f == 0.f ? 0.f : f; }  // -0 -> +0
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc)
+               : "memory");
+}
 
 __device__ __forceinline__ unsigned long long d2key(double x) {
   unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
@@ -292,45 +308,61 @@ __device__ void emit_selection(int n, int need_ties, int k, int32_t* __restrict_
   if (threadIdx.x == 0 && total != k) report(ws, kDevInternal, static_cast<unsigned>(row));
 }
 
-// float64 scores of the contract for up to four keys s[0..nk), one warp.
-// Lane j < HI forms head j's four dot products (each a sequential float64
-// chain); every lane returns the four head sums.
-__device__ __forceinline__ void rescore4(const uint16_t* __restrict__ qT,  // [DI][HI]
-                                         const float* __restrict__ w_s,    // [HI]
-                                         const uint16_t* __restrict__ k_idx, const int (&s)[4],
-                                         int nk, uint16_t* __restrict__ kst,  // [4][128] per warp
-                                         int HI, int DI, double (&x)[4]) {
+// Row data of a key for the float64 re-score: lane l holds dims 4l..4l+3.
+__device__ __forceinline__ uint2 load_key_part(const uint16_t* __restrict__ k_idx, int key, int DI) {
   const int lane = threadIdx.x & 31;
-  for (int c = lane * 8; c < 4 * DI; c += 256) {
-    const int which = c / DI;
-    const int cc = c - which * DI;
-    const int key = which < nk ? s[which] : s[0];
-    *reinterpret_cast<uint4*>(kst + which * 128 + cc) =
-        __ldg(reinterpret_cast<const uint4*>(k_idx + static_cast<int64_t>(key) * DI + cc));
+  if (lane * 4 >= DI) return make_uint2(0u, 0u);
+  return __ldg(reinterpret_cast<const uint2*>(k_idx + static_cast<int64_t>(key) * DI + lane * 4));
+}
+
+// float64 scores of the contract for two keys (one warp). raw0/raw1 are the
+// keys' row parts (load_key_part); they are widened to float64 once, into
+// this warp's kst[2][128]. Lane j < HI forms head j's two dot products, each
+// a sequential float64 chain over the dims (two dims per step); every lane
+// returns both head sums.
+__device__ __forceinline__ void rescore2(const uint16_t* __restrict__ qpad, int qstride,
+                                         const double* __restrict__ w64, uint2 raw0, uint2 raw1,
+                                         double* __restrict__ kst, int HI, int DI, double& x0,
+                                         double& x1) {
+  const int lane = threadIdx.x & 31;
+  if (lane * 4 < DI) {
+    const uint32_t w[4] = {raw0.x, raw0.y, raw1.x, raw1.y};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      double* dst = kst + e * 128 + lane * 4;
+      dst[0] = bf16_to_f64(static_cast<uint16_t>(w[2 * e] & 0xFFFFu));
+      dst[1] = bf16_to_f64(static_cast<uint16_t>(w[2 * e] >> 16));
+      dst[2] = bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] & 0xFFFFu));
+      dst[3] = bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] >> 16));
+    }
   }
   __syncwarp();
-  double r[4] = {0.0, 0.0, 0.0, 0.0};
+  double r0 = 0.0, r1 = 0.0;
   if (lane < HI) {
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-    for (int c = 0; c < DI; ++c) {
-      const double q = bf16_to_f64(qT[c * HI + lane]);
-      a0 = fma(q, bf16_to_f64(kst[c]), a0);
-      a1 = fma(q, bf16_to_f64(kst[128 + c]), a1);
-      a2 = fma(q, bf16_to_f64(kst[256 + c]), a2);
-      a3 = fma(q, bf16_to_f64(kst[384 + c]), a3);
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qpad + lane * qstride);
+    double a0 = 0.0, a1 = 0.0;
+#pragma unroll 4
+    for (int c = 0; c < DI; c += 2) {
+      const uint32_t q2 = q32[c >> 1];
+      const double qa = static_cast<double>(__uint_as_float(q2 << 16));
+      const double qb = static_cast<double>(__uint_as_float(q2 & 0xFFFF0000u));
+      const double2 k0 = *reinterpret_cast<const double2*>(kst + c);
+      const double2 k1 = *reinterpret_cast<const double2*>(kst + 128 + c);
+      a0 = fma(qa, k0.x, a0);
+      a1 = fma(qa, k1.x, a1);
+      a0 = fma(qb, k0.y, a0);
+      a1 = fma(qb, k1.y, a1);
     }
-    r[0] = a0 > 0.0 ? a0 : 0.0;
-    r[1] = a1 > 0.0 ? a1 : 0.0;
-    r[2] = a2 > 0.0 ? a2 : 0.0;
-    r[3] = a3 > 0.0 ? a3 : 0.0;
+    r0 = a0 > 0.0 ? a0 : 0.0;
+    r1 = a1 > 0.0 ? a1 : 0.0;
   }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = 0.0;
+  x0 = 0.0;
+  x1 = 0.0;
+#pragma unroll 4
   for (int j = 0; j < HI; ++j) {
-    const double w = static_cast<double>(w_s[j]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      x[e] = __dadd_rn(x[e], __dmul_rn(w, __shfl_sync(0xffffffffu, r[e], j)));
+    const double w = w64[j];
+    x0 = __dadd_rn(x0, __dmul_rn(w, __shfl_sync(0xffffffffu, r0, j)));
+    x1 = __dadd_rn(x1, __dmul_rn(w, __shfl_sync(0xffffffffu, r1, j)));
   }
   __syncwarp();
 }
@@ -350,7 +382,7 @@ struct TopkArgs {
 };
 
 template <bool kRefine>
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ Scratch sm;
   const int row = blockIdx.x;
@@ -367,13 +399,31 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   float* sc = reinterpret_cast<float*>(smem);
   int* hist = reinterpret_cast<int*>(smem + sizeof(float) * a.n_cap);
   float* cand = reinterpret_cast<float*>(hist + kBins);
+  // refine scratch after cand (see kKstExtraBytes / kQRowBytes): the q row
+  // in padded rows of DI + 2 halves
+  uint16_t* qpad = reinterpret_cast<uint16_t*>(reinterpret_cast<unsigned char*>(cand + kCandCap) +
+                                               kKstExtraBytes);
+  const int qstride = a.DI + 2;
+  const uint16_t* qrow = kRefine ? a.q_idx + static_cast<int64_t>(row) * a.HI * a.DI : nullptr;
 
-  // ---- stage the row, canonicalise -0, find its range
+  // ---- stage the row (and the query's indexer row) with asynchronous copies
   const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
-  float mn = INFINITY, mx = -INFINITY;
   const int n4 = n & ~3;
+  for (int s = threadIdx.x * 4; s < n4; s += kThreads * 4) cp_async16(sc + s, srow + s);
+  // the q row, as 32-bit words into the padded rows (while the copies fly)
+  if (kRefine) {
+    const int wpr = a.DI / 2;  // words per row
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
+    for (int e = threadIdx.x; e < a.HI * wpr; e += kThreads)
+      reinterpret_cast<uint32_t*>(qpad)[(e / wpr) * (wpr + 1) + e % wpr] = __ldg(q32 + e);
+  }
+  for (int s = n4 + threadIdx.x; s < n; s += kThreads) sc[s] = __ldg(srow + s);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  // canonicalise -0 and find the row's range
+  float mn = INFINITY, mx = -INFINITY;
   for (int s = threadIdx.x * 4; s < n4; s += kThreads * 4) {
-    float4 v = __ldg(reinterpret_cast<const float4*>(srow + s));
+    float4 v = *reinterpret_cast<const float4*>(sc + s);
     v.x = canon(v.x);
     v.y = canon(v.y);
     v.z = canon(v.z);
@@ -383,7 +433,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     mx = fmaxf(fmaxf(mx, v.x), fmaxf(fmaxf(v.y, v.z), v.w));
   }
   for (int s = n4 + threadIdx.x; s < n; s += kThreads) {
-    const float v = canon(__ldg(srow + s));
+    const float v = canon(sc[s]);
     sc[s] = v;
     mn = fminf(mn, v);
     mx = fmaxf(mx, v);
@@ -411,29 +461,41 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   // ---------------- exact float64 order: certified band + float64 re-score
   const int HI = a.HI, DI = a.DI;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* p = reinterpret_cast<unsigned char*>(cand + kCandCap);
-  uint16_t* qT = reinterpret_cast<uint16_t*>(p);  p += sizeof(uint16_t) * 32 * 128;
-  float* w_s = reinterpret_cast<float*>(p);       p += sizeof(float) * 32;
-  uint16_t* kst = reinterpret_cast<uint16_t*>(hist);  // hist/cand are free from here on
+  unsigned char* p = reinterpret_cast<unsigned char*>(qpad) + kQRowBytes;
+  int* hist256 = reinterpret_cast<int*>(p);       p += kHist256Bytes;
+  double* w64 = reinterpret_cast<double*>(p);     p += sizeof(double) * 32;
   int* tile_s = reinterpret_cast<int*>(p);        p += sizeof(int) * kThreads;
   double* tile_x = reinterpret_cast<double*>(p);  p += sizeof(double) * kThreads;
   unsigned long long* bx = reinterpret_cast<unsigned long long*>(p);
   p += sizeof(unsigned long long) * a.bcap;
   int* bidx = reinterpret_cast<int*>(p);
+  // after the select: hist + cand + extra hold the float64 key staging (2 KB per warp)
+  double* kst_all = reinterpret_cast<double*>(hist);
 
-  // A_t = sum_j |w_j| ||q_j|| (float64, rounded up by a relative slack)
-  const uint16_t* qrow = a.q_idx + static_cast<int64_t>(row) * HI * DI;
+  // A_t = sum_j |w_j| ||q_j|| (float64 from the staged row, rounded up by a
+  // relative slack); a warp takes heads warp, warp + 8, ... together
   {
-    double acc = 0.0;
-    for (int j = warp; j < HI; j += kWarps) {
-      double ss = 0.0;
-      for (int c = lane; c < DI; c += 32) {
-        const double v = bf16_to_f64(qrow[j * DI + c]);
-        ss += v * v;
-      }
+    constexpr int kHeadsPerWarp = 32 / kWarps;
+    double ss[kHeadsPerWarp];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      acc += fabs(static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + j])) * sqrt(ss);
+    for (int u = 0; u < kHeadsPerWarp; ++u) {
+      ss[u] = 0.0;
+      const int j = warp + u * kWarps;
+      if (j < HI)
+        for (int c = lane; c < DI; c += 32) {
+          const double v = bf16_to_f64(qpad[j * qstride + c]);
+          ss[u] += v * v;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < kHeadsPerWarp; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+    double acc = 0.0;
+#pragma unroll
+    for (int u = 0; u < kHeadsPerWarp; ++u) {
+      const int j = warp + u * kWarps;
+      if (j < HI) acc += fabs(static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + j])) * sqrt(ss[u]);
     }
     if (lane == 0) sm.wd[warp] = acc;
   }
@@ -445,6 +507,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   const double delta = kBoundRel * A * kmax;
   const double lo = static_cast<double>(vk) - 2.0 * delta;
   const double hi = static_cast<double>(vk) + 2.0 * delta;
+  // the same tests on float scores: f >= lo <=> f >= RU(lo), f > hi <=> f > RD(hi)
+  const float lo_f = __double2float_ru(lo);
+  const float hi_f = __double2float_rd(hi);
 
   int beg, end;
   my_segment(n, beg, end);
@@ -454,9 +519,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   __syncthreads();
   int c_in = 0, c_band = 0;
   for (int s = beg; s < end; ++s) {
-    const double f = sc[s];
-    c_in += f > hi;
-    if (f >= lo && f <= hi) {
+    const float f = sc[s];
+    c_in += f > hi_f;
+    if (f >= lo_f && f <= hi_f) {
       ++c_band;
       const int pos = atomicAdd(&sm.bc[2], 1);
       if (pos < a.bcap) bidx[pos] = s;
@@ -472,37 +537,38 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
 
   if (r == tot_band) {  // the whole band is kept: no re-score needed
     emit_selection(
-        n, 0, k, out, [&](int s) { return static_cast<double>(sc[s]) >= lo ? kAbove : kBelow; },
-        sm, a.ws, row);
+        n, 0, k, out, [&](int s) { return sc[s] >= lo_f ? kAbove : kBelow; }, sm, a.ws, row);
     return;
   }
 
-  // the query's indexer row, transposed to [c][j] so lane j reads consecutive halves
-  for (int e = threadIdx.x; e < HI * DI; e += kThreads) {
-    const int j = e / DI, c = e - j * DI;
-    qT[c * HI + j] = qrow[e];
-  }
-  if (threadIdx.x < HI) w_s[threadIdx.x] = a.w_idx[static_cast<int64_t>(row) * HI + threadIdx.x];
+  if (threadIdx.x < HI)
+    w64[threadIdx.x] = static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + threadIdx.x]);
   __syncthreads();
-  uint16_t* my_kst = kst + warp * 512;
+  double* my_kst = kst_all + warp * 256;
 
   if (tot_band <= a.bcap) {
-    // re-score the collected band, rank it by (X desc, index asc), and mark
-    // the row: kept band keys -> +inf, dropped -> -inf
-    for (int b = 4 * warp; b < tot_band; b += 4 * kWarps) {
-      const int nk = min(4, tot_band - b);
-      int ks[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ks[e] = e < nk ? bidx[b + e] : bidx[b];
-      double x[4];
-      rescore4(qT, w_s, a.k_idx, ks, nk, my_kst, HI, DI, x);
-      if (lane < nk) {
-        double mine = x[0];
-#pragma unroll
-        for (int e = 1; e < 4; ++e)
-          if (lane == e) mine = x[e];
-        bx[b + lane] = d2key(mine);
+    // re-score the collected band two keys per warp call (the next pair's rows
+    // are loaded while the current pair is scored), rank it by (X desc, index
+    // asc), and mark the row: kept band keys -> +inf, dropped -> -inf
+    int b = 2 * warp;
+    uint2 raw0 = make_uint2(0u, 0u), raw1 = make_uint2(0u, 0u);
+    if (b < tot_band) {
+      raw0 = load_key_part(a.k_idx, bidx[b], DI);
+      raw1 = load_key_part(a.k_idx, bidx[min(b + 1, tot_band - 1)], DI);
+    }
+    for (; b < tot_band; b += 2 * kWarps) {
+      const int bn = b + 2 * kWarps;
+      uint2 nraw0 = make_uint2(0u, 0u), nraw1 = make_uint2(0u, 0u);
+      if (bn < tot_band) {
+        nraw0 = load_key_part(a.k_idx, bidx[bn], DI);
+        nraw1 = load_key_part(a.k_idx, bidx[min(bn + 1, tot_band - 1)], DI);
       }
+      double x0, x1;
+      rescore2(qpad, qstride, w64, raw0, raw1, my_kst, HI, DI, x0, x1);
+      if (lane == 0) bx[b] = d2key(x0);
+      if (lane == 1 && b + 1 < tot_band) bx[b + 1] = d2key(x1);
+      raw0 = nraw0;
+      raw1 = nraw1;
     }
     __syncthreads();
     for (int b = threadIdx.x; b < tot_band; b += kThreads) {
@@ -517,8 +583,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     }
     __syncthreads();
     emit_selection(
-        n, 0, k, out, [&](int s) { return static_cast<double>(sc[s]) > hi ? kAbove : kBelow; },
-        sm, a.ws, row);
+        n, 0, k, out, [&](int s) { return sc[s] > hi_f ? kAbove : kBelow; }, sm, a.ws, row);
     return;
   }
 
@@ -529,33 +594,25 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     const int s = base + threadIdx.x;
     int flag = 0;
     if (s < n) {
-      const double f = sc[s];
-      flag = (f >= lo && f <= hi) ? 1 : 0;
+      const float f = sc[s];
+      flag = (f >= lo_f && f <= hi_f) ? 1 : 0;
     }
     unsigned long long nb64;
     const int j = static_cast<int>(block_excl_scan64(static_cast<unsigned long long>(flag), &nb64, sm));
     const int nb = static_cast<int>(nb64);
     if (flag) tile_s[j] = s;
     __syncthreads();
-    for (int jj = 4 * warp; jj < nb; jj += 4 * kWarps) {
-      const int nk = min(4, nb - jj);
-      int ks[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ks[e] = e < nk ? tile_s[jj + e] : tile_s[jj];
-      double x[4];
-      rescore4(qT, w_s, a.k_idx, ks, nk, my_kst, HI, DI, x);
-      if (lane < nk) {
-        double mine = x[0];
-#pragma unroll
-        for (int e = 1; e < 4; ++e)
-          if (lane == e) mine = x[e];
-        tile_x[jj + lane] = mine;
-      }
+    for (int jj = 2 * warp; jj < nb; jj += 2 * kWarps) {
+      const uint2 raw0 = load_key_part(a.k_idx, tile_s[jj], DI);
+      const uint2 raw1 = load_key_part(a.k_idx, tile_s[min(jj + 1, nb - 1)], DI);
+      double x0, x1;
+      rescore2(qpad, qstride, w64, raw0, raw1, my_kst, HI, DI, x0, x1);
+      if (lane == 0) tile_x[jj] = x0;
+      if (lane == 1 && jj + 1 < nb) tile_x[jj + 1] = x1;
     }
     __syncthreads();
     return nb;
   };
-  int* hist256 = reinterpret_cast<int*>(cand);  // cand is free; hist holds the staging rows
   unsigned long long pre = 0ull, msk = 0ull;
   int rr = r;
   for (int shift = 56; shift >= 0; shift -= 8) {
@@ -589,7 +646,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
       [&](int s) {
         const float v = sc[s];
         if (isnan(v)) return kTie;
-        return static_cast<double>(v) > hi ? kAbove : kBelow;
+        return v > hi_f ? kAbove : kBelow;
       },
       sm, a.ws, row);
 }
@@ -650,8 +707,8 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   size_t bytes = sizeof(float) * a.n_cap + sizeof(int) * kBins + sizeof(float) * kCandCap;
   a.bcap = 0;
   if (refine) {
-    bytes += sizeof(uint16_t) * 32 * 128 + sizeof(float) * 32 + sizeof(int) * kThreads +
-             sizeof(double) * kThreads;
+    bytes += kQRowBytes + kKstExtraBytes + kHist256Bytes + sizeof(double) * 32 +
+             sizeof(int) * kThreads + sizeof(double) * kThreads;
     if (static_cast<size_t>(max_smem) < bytes + static_bytes) return cudaErrorInvalidConfiguration;
     // band cache of up to 1,024 keys; when the row is short enough, sized so
     // that two CTAs still fit on one SM
