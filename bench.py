@@ -88,6 +88,16 @@ def barrier(world: int):
         dist.barrier()
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's synthetic chunk: every rank works on its own chunk."""
+    return seed + 1000 * rank
+
+
+def whole_job_rate(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Units per second over all ranks, for a step time that is the max over ranks."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 # ------------------------------------------------------------------- clocks
 
 
@@ -205,7 +215,7 @@ def run_ours(args):
     wl = workloads.BY_NAME[args.workload]
     d = wl.dims
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
-    x = workloads.generate(d, wl.seed + 1000 * rank, wl.kind, w_mode)
+    x = workloads.generate(d, rank_seed(wl.seed, rank), wl.kind, w_mode)
     stream = torch.cuda.current_stream()
 
     def to_dev_bf16(a):
@@ -248,7 +258,7 @@ def run_ours(args):
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
-    value = world * d.n_q / (ms_per_step / 1e3)
+    value = whole_job_rate(world, d.n_q, ms_per_step)
 
     # ---- per-kernel durations, same inputs and launch configuration
     ld = (d.ctx_len + 127) // 128 * 128
@@ -349,7 +359,7 @@ def run_ours(args):
         "pct_of_spec_bf16_peak": 100.0 * tflops / SPEC_BF16_TFLOPS,
         "useful_flop_per_step": fl["total"],
         "per_kernel_ms": per_kernel,
-        "e2e": {"value": world * d.n_q / (e2e_ms / 1e3), "unit": "queries/s",
+        "e2e": {"value": whole_job_rate(world, d.n_q, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": KERNELS_PER_LAYER * args.steps,
         "roofline": roof,
