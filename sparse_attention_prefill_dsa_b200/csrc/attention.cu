@@ -567,13 +567,11 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         }
         const bool issue_q = j == nt - 1 && q_loader && next_q;
         const bool valid = row >= 0 && row < p.ctx_len;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) x[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;
         if (!fixed_m) {
-          // per-head maximum of this tile over all 128 keys
+          // per-head maximum of this tile over all 128 keys (log2 units)
           float red[NH];
 #pragma unroll
-          for (int h = 0; h < NH; ++h) red[h] = x[h];
+          for (int h = 0; h < NH; ++h) red[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;
           const float wmax = warp_transpose_reduce<NH, true>(red);
           float* xbuf = sRed + (xc & 1) * 128;
           if (lane < NH) xbuf[sw * 32 + lane] = wmax;
@@ -632,30 +630,34 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         // the previous tile's PV has finished reading P
         ok = __all_sync(0xffffffffu, mbar_wait(p_empty, (tc & 1) ^ 1, abort_flag, p.ws, 43));
         if (!ok) break;
-        // this key's row of P: NH bf16, written as 16-byte chunks at their
-        // swizzled positions (chunk c ^ ((r >> 1) & 3) for 64-byte rows,
-        // c ^ ((r >> 2) & 1) for 32-byte rows)
-        uint32_t packed[NH / 2];
-#pragma unroll
-        for (int h2 = 0; h2 < NH / 2; ++h2) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = 2 * h2 + e;
-            pv[e] = 0.f;
-            const float mh = mrep[h];
-            if (h < H && x[h] > -INFINITY && mh > -INFINITY) pv[e] = ex2_approx(x[h] - mh);
-            lpart[h] += pv[e];
-          }
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
-          packed[h2] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
+        // this key's row of P: NH bf16, p = 2^(z scale log2e - m), written as
+        // 16-byte chunks of eight heads at their swizzled positions (chunk
+        // c ^ ((r >> 1) & 3) for 64-byte rows, c ^ ((r >> 2) & 1) for 32-byte
+        // rows); a masked key's row is zero
         unsigned char* prow = sP + r * C::kPRowBytes;
         const int swz = NH == 32 ? ((r >> 1) & 3) : ((r >> 2) & 1);
 #pragma unroll
-        for (int c = 0; c < NH / 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) =
-              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        for (int c = 0; c < NH / 8; ++c) {
+          const float4 ma = *reinterpret_cast<const float4*>(mrep + 8 * c);
+          const float4 mb = *reinterpret_cast<const float4*>(mrep + 8 * c + 4);
+          const float m8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+          uint32_t w4[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float pv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int h = 8 * c + 2 * e2 + e;
+              const float mh = m8[2 * e2 + e];
+              pv[e] = 0.f;
+              if (h < H && valid && mh > -INFINITY) pv[e] = ex2_approx(fmaf(x[h], p.scale_log2, -mh));
+              lpart[h] += pv[e];
+            }
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
+            w4[e2] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);

@@ -58,12 +58,16 @@ constexpr int kCandCap = 1024;
 constexpr int kMaxRounds = 48;
 // refine scratch: extra room that makes hist + cand + extra the float64 key
 // staging of the re-score (two keys of 128 dims per warp); the query's indexer
-// row (at most 32 x 128 bf16) in rows padded to an odd number of 32-bit words,
-// so that lane j reading row j hits bank (65 j + w) mod 32; the radix histogram
-// of the slow path
+// row (at most 32 x 128) as the high 32-bit words of its float64 values (the
+// low word of a widened bf16 is always zero), rows padded to DI + 1 words so
+// that lane j reading row j hits bank (j + c) mod 32; the radix histogram of
+// the slow path
 constexpr int kKstExtraBytes = kWarps * 2 * 128 * 8 - kBins * 4 - kCandCap * 4;
-constexpr int kQRowBytes = 32 * (128 + 2) * 2;
+constexpr int kQRowBytes = 32 * (128 + 1) * 4;
 constexpr int kHist256Bytes = 256 * 4;
+// the slow path's scratch (radix histogram, window keys and scores) overlays
+// the band cache, which that path does not use
+constexpr int kSlowScratchBytes = kHist256Bytes + 4 * kThreads + 8 * kThreads;
 static_assert(kKstExtraBytes >= 0 && kKstExtraBytes % 16 == 0, "key staging");
 
 constexpr double kDotRel = 1.0 / 32768.0;                  // 2^-15
@@ -185,9 +189,9 @@ __device__ __forceinline__ void my_segment(int n, int& beg, int& end) {
   end = min(beg + len, n);
 }
 
-// Bucket of v in [L, U]: floor((v - L) * scale), clamped to the last bucket.
-// Rounded float arithmetic is monotone in v, which is all the select needs;
-// ranges too narrow for a finite float scale use float64.
+// Bucket of v in [L, U]: (v - L) * scale rounded to an integer, clamped to the
+// last bucket. Rounded float arithmetic is monotone in v, which is all the
+// select needs; ranges too narrow for a finite float scale use float64.
 struct Bucketer {
   float Lf, scalef;
   double Ld, scaled;
@@ -202,8 +206,11 @@ struct Bucketer {
   }
   __device__ __forceinline__ int operator()(float v) const {
     if (wide) {
-      const float x = (v - Lf) * scalef;
-      return x >= static_cast<float>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
+      // round((v - L) * scale) read from the mantissa of x + 2^23 (x is in
+      // [0, kBins] up to rounding): FMA and integer pipes, no conversion
+      const float y = fmaf(v - Lf, scalef, 8388608.f);
+      const int b = __float_as_int(y) - 0x4B000000;
+      return b > kBins - 1 ? kBins - 1 : b;
     }
     const double x = (static_cast<double>(v) - Ld) * scaled;
     return x >= static_cast<double>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
@@ -318,10 +325,11 @@ __device__ __forceinline__ uint2 load_key_part(const uint16_t* __restrict__ k_id
 // float64 scores of the contract for two keys (one warp). raw0/raw1 are the
 // keys' row parts (load_key_part); they are widened to float64 once, into
 // this warp's kst[2][128]. Lane j < HI forms head j's two dot products, each
-// a sequential float64 chain over the dims (two dims per step); every lane
-// returns both head sums.
-__device__ __forceinline__ void rescore2(const uint16_t* __restrict__ qpad, int qstride,
-                                         const double* __restrict__ w64, uint2 raw0, uint2 raw1,
+// a sequential float64 chain over the dims (two dims per step), from the high
+// words of its widened q row; lane j then forms w_j * relu(dot) and the head
+// sums are added in head order. Every lane returns both sums.
+__device__ __forceinline__ void rescore2(const uint32_t* __restrict__ qhi, int qstride,
+                                         double w_lane, uint2 raw0, uint2 raw1,
                                          double* __restrict__ kst, int HI, int DI, double& x0,
                                          double& x1) {
   const int lane = threadIdx.x & 31;
@@ -337,15 +345,14 @@ __device__ __forceinline__ void rescore2(const uint16_t* __restrict__ qpad, int 
     }
   }
   __syncwarp();
-  double r0 = 0.0, r1 = 0.0;
+  double p0 = 0.0, p1 = 0.0;
   if (lane < HI) {
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qpad + lane * qstride);
+    const uint32_t* qh = qhi + lane * qstride;
     double a0 = 0.0, a1 = 0.0;
 #pragma unroll 4
     for (int c = 0; c < DI; c += 2) {
-      const uint32_t q2 = q32[c >> 1];
-      const double qa = static_cast<double>(__uint_as_float(q2 << 16));
-      const double qb = static_cast<double>(__uint_as_float(q2 & 0xFFFF0000u));
+      const double qa = __hiloint2double(static_cast<int>(qh[c]), 0);
+      const double qb = __hiloint2double(static_cast<int>(qh[c + 1]), 0);
       const double2 k0 = *reinterpret_cast<const double2*>(kst + c);
       const double2 k1 = *reinterpret_cast<const double2*>(kst + 128 + c);
       a0 = fma(qa, k0.x, a0);
@@ -353,16 +360,15 @@ __device__ __forceinline__ void rescore2(const uint16_t* __restrict__ qpad, int 
       a0 = fma(qb, k0.y, a0);
       a1 = fma(qb, k1.y, a1);
     }
-    r0 = a0 > 0.0 ? a0 : 0.0;
-    r1 = a1 > 0.0 ? a1 : 0.0;
+    p0 = __dmul_rn(w_lane, a0 > 0.0 ? a0 : 0.0);
+    p1 = __dmul_rn(w_lane, a1 > 0.0 ? a1 : 0.0);
   }
-  x0 = 0.0;
-  x1 = 0.0;
+  x0 = __dadd_rn(0.0, __shfl_sync(0xffffffffu, p0, 0));
+  x1 = __dadd_rn(0.0, __shfl_sync(0xffffffffu, p1, 0));
 #pragma unroll 4
-  for (int j = 0; j < HI; ++j) {
-    const double w = w64[j];
-    x0 = __dadd_rn(x0, __dmul_rn(w, __shfl_sync(0xffffffffu, r0, j)));
-    x1 = __dadd_rn(x1, __dmul_rn(w, __shfl_sync(0xffffffffu, r1, j)));
+  for (int j = 1; j < HI; ++j) {
+    x0 = __dadd_rn(x0, __shfl_sync(0xffffffffu, p0, j));
+    x1 = __dadd_rn(x1, __shfl_sync(0xffffffffu, p1, j));
   }
   __syncwarp();
 }
@@ -379,6 +385,8 @@ struct TopkArgs {
   WsHeader* ws;
   int n_cap;  // capacity of the score row (max row length, multiple of 4)
   int bcap;   // band cache capacity (refine only)
+  int kst_extra;  // bytes of key staging after cand: kKstExtraBytes (8 re-score warps) or 0 (4)
+  int kst_warps;  // warps that re-score band keys (8, or 4 when shared memory is short)
 };
 
 template <bool kRefine>
@@ -399,23 +407,30 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   float* sc = reinterpret_cast<float*>(smem);
   int* hist = reinterpret_cast<int*>(smem + sizeof(float) * a.n_cap);
   float* cand = reinterpret_cast<float*>(hist + kBins);
-  // refine scratch after cand (see kKstExtraBytes / kQRowBytes): the q row
-  // in padded rows of DI + 2 halves
-  uint16_t* qpad = reinterpret_cast<uint16_t*>(reinterpret_cast<unsigned char*>(cand + kCandCap) +
-                                               kKstExtraBytes);
-  const int qstride = a.DI + 2;
+  // refine scratch after cand (see kKstExtraBytes / kQRowBytes): the q row as
+  // float64 high words in padded rows of DI + 1 words
+  uint32_t* qhi = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(cand + kCandCap) +
+                                              (kRefine ? a.kst_extra : 0));
+  const int qstride = a.DI + 1;
   const uint16_t* qrow = kRefine ? a.q_idx + static_cast<int64_t>(row) * a.HI * a.DI : nullptr;
 
   // ---- stage the row (and the query's indexer row) with asynchronous copies
   const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
   const int n4 = n & ~3;
   for (int s = threadIdx.x * 4; s < n4; s += kThreads * 4) cp_async16(sc + s, srow + s);
-  // the q row, as 32-bit words into the padded rows (while the copies fly)
+  // the q row, widened to float64 once (while the copies fly); only the high
+  // words are kept
   if (kRefine) {
-    const int wpr = a.DI / 2;  // words per row
+    const int wpr = a.DI / 2;  // bf16 pairs per row
     const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
-    for (int e = threadIdx.x; e < a.HI * wpr; e += kThreads)
-      reinterpret_cast<uint32_t*>(qpad)[(e / wpr) * (wpr + 1) + e % wpr] = __ldg(q32 + e);
+    for (int e = threadIdx.x; e < a.HI * wpr; e += kThreads) {
+      const uint32_t v = __ldg(q32 + e);
+      const int j = e / wpr, c = 2 * (e - j * wpr);
+      qhi[j * qstride + c] = static_cast<uint32_t>(
+          __double2hiint(static_cast<double>(__uint_as_float(v << 16))));
+      qhi[j * qstride + c + 1] = static_cast<uint32_t>(
+          __double2hiint(static_cast<double>(__uint_as_float(v & 0xFFFF0000u))));
+    }
   }
   for (int s = n4 + threadIdx.x; s < n; s += kThreads) sc[s] = __ldg(srow + s);
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -461,16 +476,16 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   // ---------------- exact float64 order: certified band + float64 re-score
   const int HI = a.HI, DI = a.DI;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* p = reinterpret_cast<unsigned char*>(qpad) + kQRowBytes;
-  int* hist256 = reinterpret_cast<int*>(p);       p += kHist256Bytes;
-  double* w64 = reinterpret_cast<double*>(p);     p += sizeof(double) * 32;
-  int* tile_s = reinterpret_cast<int*>(p);        p += sizeof(int) * kThreads;
-  double* tile_x = reinterpret_cast<double*>(p);  p += sizeof(double) * kThreads;
-  unsigned long long* bx = reinterpret_cast<unsigned long long*>(p);
-  p += sizeof(unsigned long long) * a.bcap;
-  int* bidx = reinterpret_cast<int*>(p);
-  // after the select: hist + cand + extra hold the float64 key staging (2 KB per warp)
+  unsigned char* p = reinterpret_cast<unsigned char*>(qhi) + kQRowBytes;
+  unsigned long long* bx = reinterpret_cast<unsigned long long*>(p);   // band cache
+  int* bidx = reinterpret_cast<int*>(p + sizeof(unsigned long long) * a.bcap);
+  int* hist256 = reinterpret_cast<int*>(p);                            // slow path only
+  int* tile_s = hist256 + 256;
+  double* tile_x = reinterpret_cast<double*>(tile_s + kThreads);
+  // after the select: hist (+ cand + extra) hold the float64 key staging,
+  // 2 KB per re-scoring warp
   double* kst_all = reinterpret_cast<double*>(hist);
+  const int kw = a.kst_warps;
 
   // A_t = sum_j |w_j| ||q_j|| (float64 from the staged row, rounded up by a
   // relative slack); a warp takes heads warp, warp + 8, ... together
@@ -483,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       const int j = warp + u * kWarps;
       if (j < HI)
         for (int c = lane; c < DI; c += 32) {
-          const double v = bf16_to_f64(qpad[j * qstride + c]);
+          const double v = __hiloint2double(static_cast<int>(qhi[j * qstride + c]), 0);
           ss[u] += v * v;
         }
     }
@@ -541,30 +556,29 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     return;
   }
 
-  if (threadIdx.x < HI)
-    w64[threadIdx.x] = static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + threadIdx.x]);
-  __syncthreads();
+  const double w_lane =
+      lane < HI ? static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + lane]) : 0.0;
   double* my_kst = kst_all + warp * 256;
 
   if (tot_band <= a.bcap) {
     // re-score the collected band two keys per warp call (the next pair's rows
     // are loaded while the current pair is scored), rank it by (X desc, index
     // asc), and mark the row: kept band keys -> +inf, dropped -> -inf
-    int b = 2 * warp;
+    int b = warp < kw ? 2 * warp : tot_band;
     uint2 raw0 = make_uint2(0u, 0u), raw1 = make_uint2(0u, 0u);
     if (b < tot_band) {
       raw0 = load_key_part(a.k_idx, bidx[b], DI);
       raw1 = load_key_part(a.k_idx, bidx[min(b + 1, tot_band - 1)], DI);
     }
-    for (; b < tot_band; b += 2 * kWarps) {
-      const int bn = b + 2 * kWarps;
+    for (; b < tot_band; b += 2 * kw) {
+      const int bn = b + 2 * kw;
       uint2 nraw0 = make_uint2(0u, 0u), nraw1 = make_uint2(0u, 0u);
       if (bn < tot_band) {
         nraw0 = load_key_part(a.k_idx, bidx[bn], DI);
         nraw1 = load_key_part(a.k_idx, bidx[min(bn + 1, tot_band - 1)], DI);
       }
       double x0, x1;
-      rescore2(qpad, qstride, w64, raw0, raw1, my_kst, HI, DI, x0, x1);
+      rescore2(qhi, qstride, w_lane, raw0, raw1, my_kst, HI, DI, x0, x1);
       if (lane == 0) bx[b] = d2key(x0);
       if (lane == 1 && b + 1 < tot_band) bx[b + 1] = d2key(x1);
       raw0 = nraw0;
@@ -602,11 +616,11 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     const int nb = static_cast<int>(nb64);
     if (flag) tile_s[j] = s;
     __syncthreads();
-    for (int jj = 2 * warp; jj < nb; jj += 2 * kWarps) {
+    for (int jj = warp < kw ? 2 * warp : nb; jj < nb; jj += 2 * kw) {
       const uint2 raw0 = load_key_part(a.k_idx, tile_s[jj], DI);
       const uint2 raw1 = load_key_part(a.k_idx, tile_s[min(jj + 1, nb - 1)], DI);
       double x0, x1;
-      rescore2(qpad, qstride, w64, raw0, raw1, my_kst, HI, DI, x0, x1);
+      rescore2(qhi, qstride, w_lane, raw0, raw1, my_kst, HI, DI, x0, x1);
       if (lane == 0) tile_x[jj] = x0;
       if (lane == 1 && jj + 1 < nb) tile_x[jj + 1] = x1;
     }
@@ -706,19 +720,36 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   const size_t static_bytes = sizeof(Scratch) + 64;
   size_t bytes = sizeof(float) * a.n_cap + sizeof(int) * kBins + sizeof(float) * kCandCap;
   a.bcap = 0;
+  a.kst_extra = 0;
+  a.kst_warps = kWarps;
   if (refine) {
-    bytes += kQRowBytes + kKstExtraBytes + kHist256Bytes + sizeof(double) * 32 +
-             sizeof(int) * kThreads + sizeof(double) * kThreads;
-    if (static_cast<size_t>(max_smem) < bytes + static_bytes) return cudaErrorInvalidConfiguration;
-    // band cache of up to 1,024 keys; when the row is short enough, sized so
-    // that two CTAs still fit on one SM
-    size_t room = static_cast<size_t>(max_smem) - static_bytes - bytes;
-    const size_t half_sm = (228u * 1024u) / 2 - 2048u;
-    if (bytes + 1024 * 12 <= half_sm) room = half_sm - bytes;
+    // layout after cand: [key staging extra][q row][band cache (>= the slow
+    // path's scratch)]. Prefer two CTAs per SM with eight re-scoring warps,
+    // then one CTA per SM with eight, then one with four (no extra staging).
+    bytes += kQRowBytes;
+    const size_t min_cache = kSlowScratchBytes > 256 * 12 ? kSlowScratchBytes : 256 * 12;
+    const size_t full = static_cast<size_t>(max_smem) - static_bytes;
+    const size_t half_sm = (228u * 1024u) / 2 - 1024u - static_bytes;
+    size_t room;
+    if (bytes + kKstExtraBytes + min_cache <= half_sm) {
+      a.kst_extra = kKstExtraBytes;
+      room = half_sm - bytes - kKstExtraBytes;
+    } else if (bytes + kKstExtraBytes + min_cache <= full) {
+      a.kst_extra = kKstExtraBytes;
+      room = full - bytes - kKstExtraBytes;
+    } else if (bytes + min_cache <= full) {
+      a.kst_warps = (kBins * 4) / (2 * 128 * 8);  // the staging fits in hist alone
+      room = full - bytes;
+    } else {
+      return cudaErrorInvalidConfiguration;
+    }
     size_t bc = room / (sizeof(unsigned long long) + sizeof(int));
     if (bc > 1024) bc = 1024;
     a.bcap = static_cast<int>(bc);
-    bytes += a.bcap * (sizeof(unsigned long long) + sizeof(int));
+    bytes += a.kst_extra + a.bcap * (sizeof(unsigned long long) + sizeof(int));
+    if (bytes < static_cast<size_t>(a.kst_extra) + kQRowBytes + min_cache) {
+      return cudaErrorInvalidConfiguration;  // (unreachable: room >= min_cache)
+    }
   } else if (static_cast<size_t>(max_smem) < bytes + static_bytes) {
     return cudaErrorInvalidConfiguration;
   }
