@@ -63,7 +63,7 @@ constexpr int kMaxRounds = 48;
 // that lane j reading row j hits bank (j + c) mod 32; the radix histogram of
 // the slow path
 constexpr int kKstExtraBytes = kWarps * 2 * 128 * 8 - kBins * 4 - kCandCap * 4;
-constexpr int kQRowBytes = 32 * (128 + 1) * 4;
+constexpr int kQRowBytes = 32 * (128 + 2) * 4;
 constexpr int kHist256Bytes = 256 * 4;
 // the slow path's scratch (radix histogram, window keys and scores) overlays
 // the band cache, which that path does not use
@@ -325,51 +325,59 @@ __device__ __forceinline__ uint2 load_key_part(const uint16_t* __restrict__ k_id
 // float64 scores of the contract for two keys (one warp). raw0/raw1 are the
 // keys' row parts (load_key_part); they are widened to float64 once, into
 // this warp's kst[2][128]. Lane j < HI forms head j's two dot products, each
-// a sequential float64 chain over the dims (two dims per step), from the high
-// words of its widened q row; lane j then forms w_j * relu(dot) and the head
-// sums are added in head order. Every lane returns both sums.
-__device__ __forceinline__ void rescore2(const uint32_t* __restrict__ qhi, int qstride,
-                                         double w_lane, uint2 raw0, uint2 raw1,
-                                         double* __restrict__ kst, int HI, int DI, double& x0,
-                                         double& x1) {
+// a sequential float64 chain over the dims (fully unrolled; two dims per q
+// load from the high words of its widened q row, rows DI + 2 words apart),
+// and p = w_j * relu(dot). The products go back through kst and lanes 0 / 1
+// add them in head order. Every lane returns both sums.
+template <int DI>
+__device__ __forceinline__ void rescore2(const uint32_t* __restrict__ qhi, double w_lane,
+                                         uint2 raw0, uint2 raw1, double* __restrict__ kst, int HI,
+                                         double& x0, double& x1) {
   const int lane = threadIdx.x & 31;
   if (lane * 4 < DI) {
     const uint32_t w[4] = {raw0.x, raw0.y, raw1.x, raw1.y};
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      double* dst = kst + e * 128 + lane * 4;
-      dst[0] = bf16_to_f64(static_cast<uint16_t>(w[2 * e] & 0xFFFFu));
-      dst[1] = bf16_to_f64(static_cast<uint16_t>(w[2 * e] >> 16));
-      dst[2] = bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] & 0xFFFFu));
-      dst[3] = bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] >> 16));
+      double2* dst = reinterpret_cast<double2*>(kst + e * 128 + lane * 4);
+      dst[0] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[2 * e] & 0xFFFFu)),
+                            bf16_to_f64(static_cast<uint16_t>(w[2 * e] >> 16)));
+      dst[1] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] & 0xFFFFu)),
+                            bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] >> 16)));
     }
   }
   __syncwarp();
   double p0 = 0.0, p1 = 0.0;
   if (lane < HI) {
-    const uint32_t* qh = qhi + lane * qstride;
+    const uint2* q2 = reinterpret_cast<const uint2*>(qhi + lane * (DI + 2));
+    const double2* k0 = reinterpret_cast<const double2*>(kst);
+    const double2* k1 = reinterpret_cast<const double2*>(kst + 128);
     double a0 = 0.0, a1 = 0.0;
-#pragma unroll 4
-    for (int c = 0; c < DI; c += 2) {
-      const double qa = __hiloint2double(static_cast<int>(qh[c]), 0);
-      const double qb = __hiloint2double(static_cast<int>(qh[c + 1]), 0);
-      const double2 k0 = *reinterpret_cast<const double2*>(kst + c);
-      const double2 k1 = *reinterpret_cast<const double2*>(kst + 128 + c);
-      a0 = fma(qa, k0.x, a0);
-      a1 = fma(qa, k1.x, a1);
-      a0 = fma(qb, k0.y, a0);
-      a1 = fma(qb, k1.y, a1);
+#pragma unroll
+    for (int c2 = 0; c2 < DI / 2; ++c2) {
+      const uint2 qq = q2[c2];
+      const double qa = __hiloint2double(static_cast<int>(qq.x), 0);
+      const double qb = __hiloint2double(static_cast<int>(qq.y), 0);
+      const double2 ka = k0[c2], kb = k1[c2];
+      a0 = fma(qa, ka.x, a0);
+      a1 = fma(qa, kb.x, a1);
+      a0 = fma(qb, ka.y, a0);
+      a1 = fma(qb, kb.y, a1);
     }
     p0 = __dmul_rn(w_lane, a0 > 0.0 ? a0 : 0.0);
     p1 = __dmul_rn(w_lane, a1 > 0.0 ? a1 : 0.0);
   }
-  x0 = __dadd_rn(0.0, __shfl_sync(0xffffffffu, p0, 0));
-  x1 = __dadd_rn(0.0, __shfl_sync(0xffffffffu, p1, 0));
-#pragma unroll 4
-  for (int j = 1; j < HI; ++j) {
-    x0 = __dadd_rn(x0, __shfl_sync(0xffffffffu, p0, j));
-    x1 = __dadd_rn(x1, __shfl_sync(0xffffffffu, p1, j));
+  __syncwarp();
+  if (lane < HI) {
+    kst[lane] = p0;
+    kst[32 + lane] = p1;
   }
+  __syncwarp();
+  // lane e (mod 2) adds key e's products in head order, starting from 0
+  const double* pe = kst + (lane & 1) * 32;
+  double x = 0.0;
+  for (int j = 0; j < HI; ++j) x = __dadd_rn(x, pe[j]);
+  x0 = __shfl_sync(0xffffffffu, x, 0);
+  x1 = __shfl_sync(0xffffffffu, x, 1);
   __syncwarp();
 }
 
@@ -411,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   // float64 high words in padded rows of DI + 1 words
   uint32_t* qhi = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(cand + kCandCap) +
                                               (kRefine ? a.kst_extra : 0));
-  const int qstride = a.DI + 1;
+  const int qstride = a.DI + 2;
   const uint16_t* qrow = kRefine ? a.q_idx + static_cast<int64_t>(row) * a.HI * a.DI : nullptr;
 
   // ---- stage the row (and the query's indexer row) with asynchronous copies
@@ -578,7 +586,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
         nraw1 = load_key_part(a.k_idx, bidx[min(bn + 1, tot_band - 1)], DI);
       }
       double x0, x1;
-      rescore2(qhi, qstride, w_lane, raw0, raw1, my_kst, HI, DI, x0, x1);
+      if (DI == 128)
+        rescore2<128>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
+      else
+        rescore2<32>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
       if (lane == 0) bx[b] = d2key(x0);
       if (lane == 1 && b + 1 < tot_band) bx[b + 1] = d2key(x1);
       raw0 = nraw0;
@@ -620,7 +631,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       const uint2 raw0 = load_key_part(a.k_idx, tile_s[jj], DI);
       const uint2 raw1 = load_key_part(a.k_idx, tile_s[min(jj + 1, nb - 1)], DI);
       double x0, x1;
-      rescore2(qhi, qstride, w_lane, raw0, raw1, my_kst, HI, DI, x0, x1);
+      if (DI == 128)
+        rescore2<128>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
+      else
+        rescore2<32>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
       if (lane == 0) tile_x[jj] = x0;
       if (lane == 1 && jj + 1 < nb) tile_x[jj + 1] = x1;
     }
