@@ -6,7 +6,7 @@
 // reading this library fixes, in the spirit of the TensorFold issue #743
 // thread, whose maintainers grant no tie exception between chunkings.
 //
-// One CTA (256 threads) per query row; the row's float32 scores s = 0..t are
+// One CTA (384 threads) per query row; the row's float32 scores s = 0..t are
 // staged once in shared memory (t + 1 <= 49152 -> at most 192 KB).
 //
 // k-th largest value, exactly: a bucket select. The value range [L, U] of the
@@ -51,8 +51,9 @@
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kWarps = kThreads / 32;
+constexpr int kRescoreWarps = 8;  // warps that re-score band keys (their staging fits hist + cand + extra)
 constexpr int kBins = 2048;
 constexpr int kCandCap = 1024;
 constexpr int kMaxRounds = 48;
@@ -62,7 +63,7 @@ constexpr int kMaxRounds = 48;
 // low word of a widened bf16 is always zero), rows padded to DI + 1 words so
 // that lane j reading row j hits bank (j + c) mod 32; the radix histogram of
 // the slow path
-constexpr int kKstExtraBytes = kWarps * 2 * 128 * 8 - kBins * 4 - kCandCap * 4;
+constexpr int kKstExtraBytes = kRescoreWarps * 2 * 128 * 8 - kBins * 4 - kCandCap * 4;
 constexpr int kQRowBytes = 32 * (128 + 2) * 4;
 constexpr int kHist256Bytes = 256 * 4;
 // the slow path's scratch (radix histogram, window keys and scores) overlays
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   // A_t = sum_j |w_j| ||q_j|| (float64 from the staged row, rounded up by a
   // relative slack); a warp takes heads warp, warp + 8, ... together
   {
-    constexpr int kHeadsPerWarp = 32 / kWarps;
+    constexpr int kHeadsPerWarp = (32 + kWarps - 1) / kWarps;
     double ss[kHeadsPerWarp];
 #pragma unroll
     for (int u = 0; u < kHeadsPerWarp; ++u) {
@@ -735,7 +736,7 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   size_t bytes = sizeof(float) * a.n_cap + sizeof(int) * kBins + sizeof(float) * kCandCap;
   a.bcap = 0;
   a.kst_extra = 0;
-  a.kst_warps = kWarps;
+  a.kst_warps = kRescoreWarps;
   if (refine) {
     // layout after cand: [key staging extra][q row][band cache (>= the slow
     // path's scratch)]. Prefer two CTAs per SM with eight re-scoring warps,
