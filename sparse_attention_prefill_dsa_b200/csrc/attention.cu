@@ -46,11 +46,14 @@
 // per tile, O^T per query); the epilogue divides by the row sum, rounds to
 // bf16 and writes out / lse.
 //
-// Roles (288 threads, one CTA per SM, persistent over queries):
+// Roles (416 threads, one CTA per SM, persistent over queries):
 //   warps 0-3  producers: cp.async gathers of every tile;
 //   warp  4    TMEM owner and tcgen05.mma issuer (warp-collective, one
 //              elected lane issues);
-//   warps 5-8  softmax and epilogue (TMEM lanes 0-127 = keys, then dims); one
+//   warps 5-12 softmax and epilogue, two warps per TMEM lane quarter (lanes
+//              = keys, then dims), each on half of the heads; every softmax
+//              warp tracks the running maxima of all heads, so the decisions
+//              that need all of them are made alike without exchange. One
 //              lane also loads each query's q rows with 2D TMA once the
 //              previous query's last QK^T has completed.
 // Every wait is bounded; on a timeout the CTA records DSA_ERR_TIMEOUT, all
@@ -86,7 +89,10 @@ struct AttnCfg {
   static constexpr int kPBytes = kKeys * kPRowBytes;
   static constexpr uint32_t kPSwz = NH == 32 ? 4u : 6u;  // descriptor code: 64B / 32B swizzle
   static constexpr int kProducerThreads = 128;        // warps 0-3
-  static constexpr int kThreads = 288;
+  static constexpr int kSoftmaxWarps = 8;            // two per TMEM lane quarter, half the heads each
+  static constexpr int HH = NH / 2;                   // heads per softmax warp
+  static constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+  static constexpr int kThreads = 32 * (5 + kSoftmaxWarps);
   static constexpr int kRowsPerThread = kKeys / 16;   // keys 32w + lane/8 + 4i, i < 8
   static constexpr uint32_t kQBytes = H * 128 * kQChunks;  // q boxes (zero-filled past Dc+Dr)
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, NH, false, false);
@@ -102,10 +108,10 @@ struct AttnCfg {
   static constexpr int kOffRope = kOffPairs + kPairs * kPairBytes;
   static constexpr int kOffQ = kOffRope + kChunkBytes;
   static constexpr int kOffP = kOffQ + kQChunks * kQChunkBytes;
-  static constexpr int kOffRed = kOffP + kPBytes;                // [2][4][32] floats
-  static constexpr int kOffNorm = kOffRed + 2 * 4 * 32 * 4;      // [4][32] floats
-  static constexpr int kOffM = kOffNorm + 4 * 32 * 4;            // [4 warps][32] floats
-  static constexpr int kOffBar = kOffM + 4 * 32 * 4;
+  static constexpr int kOffRed = kOffP + kPBytes;                // [2][8 warps][16] floats
+  static constexpr int kOffNorm = kOffRed + 2 * 8 * 16 * 4;      // [8 warps][32] floats
+  static constexpr int kOffM = kOffNorm + 8 * 32 * 4;            // [8 warps][32] floats
+  static constexpr int kOffBar = kOffM + 8 * 32 * 4;
   static constexpr int kNumBars = 3 * kPairs + 17;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
@@ -175,36 +181,26 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV]) {
   return v[0];
 }
 
-template <int NH>
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&x)[NH]) {
-  if constexpr (NH == 32) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr, r);
-    tmem_ld_wait();
+// A warp's 32 TMEM lanes x NC consecutive 32-bit columns (NC = 8, 16 or 32).
+template <int NC>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&x)[NC]) {
+  uint32_t r[NC];
+  if constexpr (NC == 32) tmem_ld_32x32b_x32(taddr, r);
+  else if constexpr (NC == 16) tmem_ld_32x32b_x16(taddr, r);
+  else tmem_ld_32x32b_x8(taddr, r);
+  tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
-  } else {
-    uint32_t r[16];
-    tmem_ld_32x32b_x16(taddr, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(r[e]);
-  }
+  for (int e = 0; e < NC; ++e) x[e] = __uint_as_float(r[e]);
 }
 
-template <int NH>
-__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&x)[NH]) {
-  if constexpr (NH == 32) {
-    uint32_t r[32];
+template <int NC>
+__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&x)[NC]) {
+  uint32_t r[NC];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(x[e]);
-    tmem_st_32x32b_x32(taddr, r);
-  } else {
-    uint32_t r[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(x[e]);
-    tmem_st_32x32b_x16(taddr, r);
-  }
+  for (int e = 0; e < NC; ++e) r[e] = __float_as_uint(x[e]);
+  if constexpr (NC == 32) tmem_st_32x32b_x32(taddr, r);
+  else if constexpr (NC == 16) tmem_st_32x32b_x16(taddr, r);
+  else tmem_st_32x32b_x8(taddr, r);
 }
 
 // Shared-memory descriptor advanced by a byte offset (the start address is
@@ -344,12 +340,12 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     mbar_init(q_full, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 128);
+      mbar_init(&s_empty[b], C::kSoftmaxThreads);
       mbar_init(&o_full[b], 1);
-      mbar_init(&o_empty[b], 128);
-      mbar_init(&exch[b], 128);
+      mbar_init(&o_empty[b], C::kSoftmaxThreads);
+      mbar_init(&exch[b], C::kSoftmaxThreads);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, C::kSoftmaxThreads);
     mbar_init(p_empty, 1);
     mbar_init(o_step, 1);
     mbar_init(mma_done, 1);
@@ -495,9 +491,11 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     drain_wait(mma_done, 0);
   } else {
     // ------------------------------------------------- softmax and epilogue
+    constexpr int HH = C::HH;
     const int quarter = warp & 3;               // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;          // key lane (and dim lane in the epilogue)
-    const int sw = warp - 5;                    // softmax warp index 0..3
+    const int sw = warp - 5;                    // softmax warp index 0..7
+    const int hh = sw >> 2;                     // this warp's heads: hh*HH .. hh*HH+HH-1
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const bool q_loader = warp == 5 && lane == 0;
     int q_loads = 0;
@@ -514,19 +512,22 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     // max_s ||k_s|| of the context, with the rounding slack of its float32 sum
     const float kmax = __uint_as_float(*reinterpret_cast<volatile unsigned int*>(&p.ws->akmax_bits));
     const float bound_scale = fabsf(p.scale_log2) * kmax;
+    // the exchange slot of head h (lane) from the warp of quarter-rank qq of
+    // h's half: warps hh*4 .. hh*4+3 hold the halves' partial values
+    const int xslot = (lane / HH) * 4 * 16 + (lane % HH);
     for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
       const int nt = n_tiles_of(p, i);
       const int ob = qi & 1;
       const bool next_q = i + static_cast<int>(gridDim.x) < p.n_q;
-      float m_lane = -INFINITY;       // running max (log2 units) of head `lane`
+      float m_lane = -INFINITY;       // running max (log2 units) of head `lane` (all heads)
       float bound_lane = INFINITY;    // B_lane: bound on every score of head `lane`
       bool fixed_m = false;           // B_h <= m_h + 64 for every head: keep m as it is
       float* mrep = sM + sw * 32;     // running max of every head (this warp's copy)
-      float lpart[NH];                // this key lane's share of the row sums
+      float lpart[HH];                // this key lane's share of the row sums of its heads
       mrep[lane] = -INFINITY;
       __syncwarp();
 #pragma unroll
-      for (int h = 0; h < NH; ++h) lpart[h] = 0.f;
+      for (int h = 0; h < HH; ++h) lpart[h] = 0.f;
       for (int j = 0; j < nt; ++j, ++tc) {
         const int sb = tc & 1;
         const int row = row_next;
@@ -538,18 +539,18 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (tc >> 1) & 1, abort_flag, p.ws, 40));
         if (!ok) break;
         tc_fence_after();
-        float x[NH];
-        tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemS + sb * NH, x);
+        float x[HH];
+        tmem_ld_row<HH>(tmem_base + lane_addr + C::kTmemS + sb * NH + hh * HH, x);
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
         if (j == 0) {
-          // this warp's share of ||q_h||^2 (q chunks sw, sw+4, ...; lane = head),
-          // reading the 16-byte units of a row in a lane-rotated order
+          // this warp's share of ||q_h||^2 for every head (q chunks sw, sw+8;
+          // lane = head), reading a row's 16-byte units in a lane-rotated order
           ok = __all_sync(0xffffffffu, mbar_wait(q_full, qi & 1, abort_flag, p.ws, 46));
           if (!ok) break;
           float qn2 = 0.f;
           if (lane < NH) {
-            for (int c = sw; c < C::kQChunks; c += 4) {
+            for (int c = sw; c < C::kQChunks; c += C::kSoftmaxWarps) {
               const unsigned char* qrow = sQ + c * C::kQChunkBytes + lane * 128;
 #pragma unroll
               for (int u = 0; u < 8; ++u) {
@@ -562,28 +563,31 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
                 }
               }
             }
-            sNorm[sw * 32 + lane] = qn2;
           }
+          sNorm[sw * 32 + lane] = qn2;
         }
         const bool issue_q = j == nt - 1 && q_loader && next_q;
         const bool valid = row >= 0 && row < p.ctx_len;
         if (!fixed_m) {
           // per-head maximum of this tile over all 128 keys (log2 units)
-          float red[NH];
+          float red[HH];
 #pragma unroll
-          for (int h = 0; h < NH; ++h) red[h] = (valid && h < H) ? x[h] * p.scale_log2 : -INFINITY;
-          const float wmax = warp_transpose_reduce<NH, true>(red);
+          for (int h = 0; h < HH; ++h)
+            red[h] = (valid && hh * HH + h < H) ? x[h] * p.scale_log2 : -INFINITY;
+          const float wmax = warp_transpose_reduce<HH, true>(red);
           float* xbuf = sRed + (xc & 1) * 128;
-          if (lane < NH) xbuf[sw * 32 + lane] = wmax;
+          if (lane < HH) xbuf[sw * 16 + lane] = wmax;
           mbar_arrive(&exch[xc & 1]);
           ok = __all_sync(0xffffffffu, mbar_wait(&exch[xc & 1], (xc >> 1) & 1, abort_flag, p.ws, 41));
           ++xc;
           if (!ok) break;
           float tmax = -INFINITY;
           if (lane < NH)
-            tmax = fmaxf(fmaxf(xbuf[lane], xbuf[32 + lane]), fmaxf(xbuf[64 + lane], xbuf[96 + lane]));
+            tmax = fmaxf(fmaxf(xbuf[xslot], xbuf[xslot + 16]), fmaxf(xbuf[xslot + 32], xbuf[xslot + 48]));
           if (j == 0 && lane < NH) {
-            const float qn2 = sNorm[lane] + sNorm[32 + lane] + sNorm[64 + lane] + sNorm[96 + lane];
+            float qn2 = 0.f;
+#pragma unroll
+            for (int w = 0; w < C::kSoftmaxWarps; ++w) qn2 += sNorm[w * 32 + lane];
             // the float32 sums are within 2^-8 of exact; the slack covers them
             bound_lane = bound_scale * sqrtf(qn2) * (1.f + 0.00390625f);
           }
@@ -592,26 +596,26 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             const float m_new = fmaxf(m_lane, tmax);
             const float alpha_lane = m_lane == -INFINITY ? 0.f : ex2_approx(m_lane - m_new);
             m_lane = m_new;
-            float alpha[NH];
+            float alpha[HH];
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-              alpha[h] = __shfl_sync(0xffffffffu, alpha_lane, h);
+            for (int h = 0; h < HH; ++h) {
+              alpha[h] = __shfl_sync(0xffffffffu, alpha_lane, hh * HH + h);
               lpart[h] *= alpha[h];
             }
             mrep[lane] = m_lane;
             __syncwarp();
-            if (j > 0) {  // rescale O^T once the previous tile's PV is complete
+            if (j > 0) {  // rescale this warp's O^T columns once the previous tile's PV is complete
               ok = __all_sync(0xffffffffu, mbar_wait(o_step, (tc - 1) & 1, abort_flag, p.ws, 42));
               if (!ok) break;
               tc_fence_after();
 #pragma unroll 1
               for (int mb = 0; mb < C::MB; ++mb) {
-                const uint32_t ta = tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH;
-                float o[NH];
-                tmem_ld_row<NH>(ta, o);
+                const uint32_t ta = tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH + hh * HH;
+                float o[HH];
+                tmem_ld_row<HH>(ta, o);
 #pragma unroll
-                for (int h = 0; h < NH; ++h) o[h] *= alpha[h];
-                tmem_st_row<NH>(ta, o);
+                for (int h = 0; h < HH; ++h) o[h] *= alpha[h];
+                tmem_st_row<HH>(ta, o);
               }
               tmem_st_wait();
             }
@@ -630,14 +634,15 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         // the previous tile's PV has finished reading P
         ok = __all_sync(0xffffffffu, mbar_wait(p_empty, (tc & 1) ^ 1, abort_flag, p.ws, 43));
         if (!ok) break;
-        // this key's row of P: NH bf16, p = 2^(z scale log2e - m), written as
-        // 16-byte chunks of eight heads at their swizzled positions (chunk
-        // c ^ ((r >> 1) & 3) for 64-byte rows, c ^ ((r >> 2) & 1) for 32-byte
-        // rows); a masked key's row is zero
+        // this key's P for this warp's heads: p = 2^(z scale log2e - m) as bf16,
+        // written as 16-byte chunks of eight heads at their swizzled positions
+        // (chunk c ^ ((r >> 1) & 3) for 64-byte rows, c ^ ((r >> 2) & 1) for
+        // 32-byte rows); a masked key's row is zero
         unsigned char* prow = sP + r * C::kPRowBytes;
         const int swz = NH == 32 ? ((r >> 1) & 3) : ((r >> 2) & 1);
 #pragma unroll
-        for (int c = 0; c < NH / 8; ++c) {
+        for (int cl = 0; cl < HH / 8; ++cl) {
+          const int c = hh * (HH / 8) + cl;  // chunk of heads 8c .. 8c+7
           const float4 ma = *reinterpret_cast<const float4*>(mrep + 8 * c);
           const float4 mb = *reinterpret_cast<const float4*>(mrep + 8 * c + 4);
           const float m8[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
@@ -647,11 +652,12 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             float pv[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int h = 8 * c + 2 * e2 + e;
+              const int hl = 8 * cl + 2 * e2 + e;  // local head
               const float mh = m8[2 * e2 + e];
               pv[e] = 0.f;
-              if (h < H && valid && mh > -INFINITY) pv[e] = ex2_approx(fmaf(x[h], p.scale_log2, -mh));
-              lpart[h] += pv[e];
+              if (8 * c + 2 * e2 + e < H && valid && mh > -INFINITY)
+                pv[e] = ex2_approx(fmaf(x[hl], p.scale_log2, -mh));
+              lpart[hl] += pv[e];
             }
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
             w4[e2] = *reinterpret_cast<const uint32_t*>(&b2);
@@ -667,31 +673,32 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&o_full[ob], (qi >> 1) & 1, abort_flag, p.ws, 44));
       if (!ok) break;
       tc_fence_after();
-      const float lsum = warp_transpose_reduce<NH, false>(lpart);
+      const float lsum = warp_transpose_reduce<HH, false>(lpart);
       float* xbuf = sRed + (xc & 1) * 128;
-      if (lane < NH) xbuf[sw * 32 + lane] = lsum;
+      if (lane < HH) xbuf[sw * 16 + lane] = lsum;
       mbar_arrive(&exch[xc & 1]);
       ok = __all_sync(0xffffffffu, mbar_wait(&exch[xc & 1], (xc >> 1) & 1, abort_flag, p.ws, 45));
       ++xc;
       if (!ok) break;
       float l_lane = 0.f;
-      if (lane < NH) l_lane = xbuf[lane] + xbuf[32 + lane] + xbuf[64 + lane] + xbuf[96 + lane];
+      if (lane < NH) l_lane = xbuf[xslot] + xbuf[xslot + 16] + xbuf[xslot + 32] + xbuf[xslot + 48];
       const float inv_lane = l_lane > 0.f ? 1.f / l_lane : 0.f;
       if (sw == 0 && lane < H && p.lse)
         p.lse[static_cast<int64_t>(i) * H + lane] =
             l_lane > 0.f ? (m_lane + log2f(l_lane)) * 0.6931471805599453f : -INFINITY;
-      float inv[NH];
+      float inv[HH];
 #pragma unroll
-      for (int h = 0; h < NH; ++h) inv[h] = __shfl_sync(0xffffffffu, inv_lane, h);
+      for (int h = 0; h < HH; ++h) inv[h] = __shfl_sync(0xffffffffu, inv_lane, hh * HH + h);
 #pragma unroll 1
       for (int mb = 0; mb < C::MB; ++mb) {
-        float o[NH];
-        tmem_ld_row<NH>(tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH, o);
+        float o[HH];
+        tmem_ld_row<HH>(tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH + hh * HH, o);
         const int d = mb * 128 + r;
         if (d < DC) {
-          uint16_t* orow = p.out + static_cast<int64_t>(i) * H * DC + d;
+          uint16_t* orow = p.out + (static_cast<int64_t>(i) * H + hh * HH) * DC + d;
 #pragma unroll
-          for (int h = 0; h < H; ++h) orow[h * DC] = f32_to_bf16_rne(o[h] * inv[h]);
+          for (int h = 0; h < HH; ++h)
+            if (hh * HH + h < H) orow[h * DC] = f32_to_bf16_rne(o[h] * inv[h]);
         }
       }
       tc_fence_before();
