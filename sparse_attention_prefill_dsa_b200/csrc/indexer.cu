@@ -203,40 +203,47 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t it = 0, uq = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        int qb, kt0, kt1;
-        if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
-        if (!(ok = mbar_wait(q_full, uq & 1, abort_flag, p.ws, 4))) break;
-        for (int kt = kt0; kt < kt1; ++kt, ++it) {
-          const int st = it % C::kStages, buf = it & 1;
-          if (!(ok = mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, abort_flag, p.ws, 5))) break;
-          if (!(ok = mbar_wait(&k_full[st], (it / C::kStages) & 1, abort_flag, p.ws, 6))) break;
-          tc_fence_after();
-          const uint32_t d = tmem_base + buf * C::kN;
-          const uint32_t k_addr = smem_u32(sK + st * C::kKTileBytes);
-          const uint32_t q_addr = smem_u32(sQ);
+    // The whole warp runs the loop with warp-uniform operands and one elected
+    // lane issues: descriptors are a base plus compile-time offsets, so an
+    // issue costs a few cycles (a single-thread loop with run-time
+    // descriptors costs more than a 128-cycle MMA).
+    uint32_t it = 0, uq = 0;
+    bool ok = true;
+    const uint64_t dk0 = smem_desc(smem_u32(sK), 16, C::kSbo, C::kSwzCode);
+    const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, C::kSbo, C::kSwzCode);
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      int qb, kt0, kt1;
+      if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full, uq & 1, abort_flag, p.ws, 4)))) break;
+      for (int kt = kt0; kt < kt1; ++kt, ++it) {
+        const int st = it % C::kStages, buf = it & 1;
+        if (!(ok = __all_sync(0xffffffffu,
+                              mbar_wait(&acc_empty[buf], ((it >> 1) & 1) ^ 1, abort_flag, p.ws, 5))))
+          break;
+        if (!(ok = __all_sync(0xffffffffu,
+                              mbar_wait(&k_full[st], (it / C::kStages) & 1, abort_flag, p.ws, 6))))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * C::kN;
+        const uint64_t dk = dk0 + static_cast<uint64_t>((st * C::kKTileBytes) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < C::kKSteps; ++ks) {
-            const int c = ks / C::kStepsPerChunk;
-            const uint32_t off = (ks % C::kStepsPerChunk) * 32;
-            const uint64_t a = smem_desc(k_addr + c * C::kKChunkBytes + off, 16, C::kSbo, C::kSwzCode);
-            const uint64_t b = smem_desc(q_addr + c * C::kQChunkBytes + off, 16, C::kSbo, C::kSwzCode);
-            mma_bf16_ss(d, a, b, C::kIdesc, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(&k_empty[st]);
-          mma_commit(&acc_full[buf]);
+        for (int ks = 0; ks < C::kKSteps; ++ks) {
+          const int c = ks / C::kStepsPerChunk;
+          const uint32_t off = (ks % C::kStepsPerChunk) * 32;
+          const uint64_t a = dk + static_cast<uint64_t>((c * C::kKChunkBytes + off) >> 4);
+          const uint64_t b = dq0 + static_cast<uint64_t>((c * C::kQChunkBytes + off) >> 4);
+          mma_bf16_ss_warp(d, a, b, C::kIdesc, ks > 0 ? 1u : 0u);
         }
-        if (!ok) break;
-        mma_commit(q_empty);
-        ++uq;
+        mma_commit_warp(&k_empty[st]);
+        mma_commit_warp(&acc_full[buf]);
       }
-      // every MMA issued must complete before TMEM is released
-      mma_commit(mma_done);
-      drain_wait(mma_done, 0);
+      if (!ok) break;
+      mma_commit_warp(q_empty);
+      ++uq;
     }
+    // every MMA issued must complete before TMEM is released
+    mma_commit_warp(mma_done);
+    drain_wait(mma_done, 0);
   } else {
     // ------------------------------------------------------------ epilogue
     const int wg = (warp - 2) >> 2;        // column half
