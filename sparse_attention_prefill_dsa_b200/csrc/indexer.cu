@@ -266,20 +266,36 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int s = kt * C::kM + key_local;
+        // two 32-column groups per TMEM wait; the weights of a group are read
+        // as float4 broadcasts
 #pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
-          const int col0 = wg * 128 + g * 32;
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + col0, v);
+        for (int g2 = 0; g2 < 2; ++g2) {
+          uint32_t v[2][32];
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + (2 * g2 + h) * 32, v[h]);
           tmem_ld_wait();
 #pragma unroll
-          for (int qq = 0; qq < 32 / HI; ++qq) {
-            float acc = 0.f;
+          for (int h = 0; h < 2; ++h) {
+            const int col0 = wg * 128 + (2 * g2 + h) * 32;
+            float wv[32];
 #pragma unroll
-            for (int j = 0; j < HI; ++j)
-              acc = fmaf(w[col0 + qq * HI + j], fmaxf(__uint_as_float(v[qq * HI + j]), 0.f), acc);
-            const int i = qb * C::kQB + (col0 + qq * HI) / HI;
-            if (i < p.n_q && s <= p.q_pos0 + i) p.scores[static_cast<int64_t>(i) * p.ld + s] = acc;
+            for (int e = 0; e < 8; ++e) {
+              const float4 w4 = *reinterpret_cast<const float4*>(w + col0 + 4 * e);
+              wv[4 * e] = w4.x;
+              wv[4 * e + 1] = w4.y;
+              wv[4 * e + 2] = w4.z;
+              wv[4 * e + 3] = w4.w;
+            }
+#pragma unroll
+            for (int qq = 0; qq < 32 / HI; ++qq) {
+              float acc = 0.f;
+#pragma unroll
+              for (int j = 0; j < HI; ++j)
+                acc = fmaf(wv[qq * HI + j], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f), acc);
+              const int i = qb * C::kQB + (col0 + qq * HI) / HI;
+              if (i < p.n_q && s <= p.q_pos0 + i) p.scores[static_cast<int64_t>(i) * p.ld + s] = acc;
+            }
           }
         }
         tc_fence_before();
