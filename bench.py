@@ -42,7 +42,9 @@ L2_FLUSH_BYTES = 256 << 20
 # named beside each entry; traffic scales with the query count (q rows, outputs,
 # index rows), so a launch's traffic is this figure times n_q. An entry is
 # removed whenever its kernel changes after the capture.
-PROFILED_DRAM_BYTES_PER_QUERY = {}
+PROFILED_DRAM_BYTES_PER_QUERY = {
+    "sparse_attn": (141.63e6 / 2048, "profiles/sparse_attn_tc_chunk2k_ctx8k.md"),
+}
 
 KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
 
