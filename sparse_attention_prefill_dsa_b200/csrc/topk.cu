@@ -57,14 +57,15 @@ constexpr int kRescoreWarps = 8;  // warps that re-score band keys (their stagin
 constexpr int kBins = 2048;
 constexpr int kCandCap = 1024;
 constexpr int kMaxRounds = 48;
-// refine scratch: extra room that makes hist + cand + extra the float64 key
-// staging of the re-score (two keys of 128 dims per warp); the query's indexer
-// row (at most 32 x 128) as the high 32-bit words of its float64 values (the
-// low word of a widened bf16 is always zero), rows padded to DI + 1 words so
-// that lane j reading row j hits bank (j + c) mod 32; the radix histogram of
-// the slow path
-constexpr int kKstExtraBytes = kRescoreWarps * 2 * 128 * 8 - kBins * 4 - kCandCap * 4;
-constexpr int kQRowBytes = 32 * (128 + 2) * 4;
+// refine scratch: extra room that makes hist + cand + extra the key staging of
+// the re-score (four keys of 128 dims as float64 high words, 2 KB per warp);
+// the query's indexer row (at most 32 x 128) as the high 32-bit words of its
+// float64 values (the low word of a widened bf16 is always zero), rows padded
+// to DI + 4 words so that the 16-byte loads of lanes j .. j+7 (row j, same
+// column) cover all 32 banks; the radix histogram of the slow path
+constexpr int kKstStageBytes = 4 * 128 * 4;
+constexpr int kKstExtraBytes = kRescoreWarps * kKstStageBytes - kBins * 4 - kCandCap * 4;
+constexpr int kQRowBytes = 32 * (128 + 4) * 4;
 constexpr int kHist256Bytes = 256 * 4;
 // the slow path's scratch (radix histogram, window keys and scores) overlays
 // the band cache, which that path does not use
@@ -323,63 +324,75 @@ __device__ __forceinline__ uint2 load_key_part(const uint16_t* __restrict__ k_id
   return __ldg(reinterpret_cast<const uint2*>(k_idx + static_cast<int64_t>(key) * DI + lane * 4));
 }
 
-// float64 scores of the contract for two keys (one warp). raw0/raw1 are the
-// keys' row parts (load_key_part); they are widened to float64 once, into
-// this warp's kst[2][128]. Lane j < HI forms head j's two dot products, each
-// a sequential float64 chain over the dims (fully unrolled; two dims per q
-// load from the high words of its widened q row, rows DI + 2 words apart),
-// and p = w_j * relu(dot). The products go back through kst and lanes 0 / 1
-// add them in head order. Every lane returns both sums.
+// float64 scores of the contract for four keys (one warp). raw[e] is key e's
+// row part (load_key_part); lanes widen it once into this warp's kst as the
+// high 32-bit words of the float64 values ([4][128] words; the low word of a
+// widened bf16 is zero). Lane j < HI forms head j's four dot products, each a
+// sequential float64 chain over the dims (fully unrolled; four dims per
+// 16-byte load of the q row's high words, rows DI + 4 words apart, and four
+// per broadcast load of each key), and p = w_j * relu(dot). The products go
+// back through kst ([4][34] doubles) and lane e < 4 adds key e's in head
+// order and returns that sum (other lanes return 0).
 template <int DI>
-__device__ __forceinline__ void rescore2(const uint32_t* __restrict__ qhi, double w_lane,
-                                         uint2 raw0, uint2 raw1, double* __restrict__ kst, int HI,
-                                         double& x0, double& x1) {
+__device__ __forceinline__ double rescore4(const uint32_t* __restrict__ qhi, double w_lane,
+                                           const uint2 (&raw)[4], uint32_t* __restrict__ kst, int HI) {
   const int lane = threadIdx.x & 31;
   if (lane * 4 < DI) {
-    const uint32_t w[4] = {raw0.x, raw0.y, raw1.x, raw1.y};
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      double2* dst = reinterpret_cast<double2*>(kst + e * 128 + lane * 4);
-      dst[0] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[2 * e] & 0xFFFFu)),
-                            bf16_to_f64(static_cast<uint16_t>(w[2 * e] >> 16)));
-      dst[1] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] & 0xFFFFu)),
-                            bf16_to_f64(static_cast<uint16_t>(w[2 * e + 1] >> 16)));
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t w[2] = {raw[e].x, raw[e].y};
+      uint32_t h[4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        h[2 * u] = static_cast<uint32_t>(__double2hiint(bf16_to_f64(static_cast<uint16_t>(w[u] & 0xFFFFu))));
+        h[2 * u + 1] = static_cast<uint32_t>(__double2hiint(bf16_to_f64(static_cast<uint16_t>(w[u] >> 16))));
+      }
+      *reinterpret_cast<uint4*>(kst + e * 128 + lane * 4) = make_uint4(h[0], h[1], h[2], h[3]);
     }
   }
   __syncwarp();
-  double p0 = 0.0, p1 = 0.0;
+  double pr[4] = {0.0, 0.0, 0.0, 0.0};
   if (lane < HI) {
-    const uint2* q2 = reinterpret_cast<const uint2*>(qhi + lane * (DI + 2));
-    const double2* k0 = reinterpret_cast<const double2*>(kst);
-    const double2* k1 = reinterpret_cast<const double2*>(kst + 128);
-    double a0 = 0.0, a1 = 0.0;
+    const uint4* q4 = reinterpret_cast<const uint4*>(qhi + lane * (DI + 4));
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int c2 = 0; c2 < DI / 2; ++c2) {
-      const uint2 qq = q2[c2];
-      const double qa = __hiloint2double(static_cast<int>(qq.x), 0);
-      const double qb = __hiloint2double(static_cast<int>(qq.y), 0);
-      const double2 ka = k0[c2], kb = k1[c2];
-      a0 = fma(qa, ka.x, a0);
-      a1 = fma(qa, kb.x, a1);
-      a0 = fma(qb, ka.y, a0);
-      a1 = fma(qb, kb.y, a1);
+    for (int c4 = 0; c4 < DI / 4; ++c4) {
+      const uint4 qq = q4[c4];
+      const double qd[4] = {__hiloint2double(static_cast<int>(qq.x), 0), __hiloint2double(static_cast<int>(qq.y), 0),
+                            __hiloint2double(static_cast<int>(qq.z), 0), __hiloint2double(static_cast<int>(qq.w), 0)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint4 kk = reinterpret_cast<const uint4*>(kst + e * 128)[c4];
+        acc[e] = fma(qd[0], __hiloint2double(static_cast<int>(kk.x), 0), acc[e]);
+        acc[e] = fma(qd[1], __hiloint2double(static_cast<int>(kk.y), 0), acc[e]);
+        acc[e] = fma(qd[2], __hiloint2double(static_cast<int>(kk.z), 0), acc[e]);
+        acc[e] = fma(qd[3], __hiloint2double(static_cast<int>(kk.w), 0), acc[e]);
+      }
     }
-    p0 = __dmul_rn(w_lane, a0 > 0.0 ? a0 : 0.0);
-    p1 = __dmul_rn(w_lane, a1 > 0.0 ? a1 : 0.0);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[e] = __dmul_rn(w_lane, acc[e] > 0.0 ? acc[e] : 0.0);
   }
   __syncwarp();
+  double* prod = reinterpret_cast<double*>(kst);
   if (lane < HI) {
-    kst[lane] = p0;
-    kst[32 + lane] = p1;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) prod[e * 34 + lane] = pr[e];
   }
   __syncwarp();
-  // lane e (mod 2) adds key e's products in head order, starting from 0
-  const double* pe = kst + (lane & 1) * 32;
-  double x = 0.0;
-  for (int j = 0; j < HI; ++j) x = __dadd_rn(x, pe[j]);
-  x0 = __shfl_sync(0xffffffffu, x, 0);
-  x1 = __shfl_sync(0xffffffffu, x, 1);
+  double sum = 0.0;
+  if (lane < 4) {
+    const double2* pe = reinterpret_cast<const double2*>(prod + lane * 34);
+#pragma unroll
+    for (int j2 = 0; j2 < 16; ++j2) {
+      if (2 * j2 < HI) {
+        const double2 v = pe[j2];
+        sum = __dadd_rn(sum, v.x);
+        sum = __dadd_rn(sum, v.y);  // HI is even
+      }
+    }
+  }
   __syncwarp();
+  return sum;
 }
 
 struct TopkArgs {
@@ -417,10 +430,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   int* hist = reinterpret_cast<int*>(smem + sizeof(float) * a.n_cap);
   float* cand = reinterpret_cast<float*>(hist + kBins);
   // refine scratch after cand (see kKstExtraBytes / kQRowBytes): the q row as
-  // float64 high words in padded rows of DI + 1 words
+  // float64 high words in padded rows of DI + 4 words
   uint32_t* qhi = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(cand + kCandCap) +
                                               (kRefine ? a.kst_extra : 0));
-  const int qstride = a.DI + 2;
+  const int qstride = a.DI + 4;
   const uint16_t* qrow = kRefine ? a.q_idx + static_cast<int64_t>(row) * a.HI * a.DI : nullptr;
 
   // ---- stage the row (and the query's indexer row) with asynchronous copies
@@ -491,9 +504,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   int* hist256 = reinterpret_cast<int*>(p);                            // slow path only
   int* tile_s = hist256 + 256;
   double* tile_x = reinterpret_cast<double*>(tile_s + kThreads);
-  // after the select: hist (+ cand + extra) hold the float64 key staging,
+  // after the select: hist (+ cand + extra) hold the re-score's key staging,
   // 2 KB per re-scoring warp
-  double* kst_all = reinterpret_cast<double*>(hist);
+  uint32_t* kst_all = reinterpret_cast<uint32_t*>(hist);
   const int kw = a.kst_warps;
 
   // A_t = sum_j |w_j| ||q_j|| (float64 from the staged row, rounded up by a
@@ -567,34 +580,29 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   const double w_lane =
       lane < HI ? static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + lane]) : 0.0;
-  double* my_kst = kst_all + warp * 256;
+  uint32_t* my_kst = kst_all + warp * 512;
 
   if (tot_band <= a.bcap) {
-    // re-score the collected band two keys per warp call (the next pair's rows
-    // are loaded while the current pair is scored), rank it by (X desc, index
-    // asc), and mark the row: kept band keys -> +inf, dropped -> -inf
-    int b = warp < kw ? 2 * warp : tot_band;
-    uint2 raw0 = make_uint2(0u, 0u), raw1 = make_uint2(0u, 0u);
-    if (b < tot_band) {
-      raw0 = load_key_part(a.k_idx, bidx[b], DI);
-      raw1 = load_key_part(a.k_idx, bidx[min(b + 1, tot_band - 1)], DI);
-    }
-    for (; b < tot_band; b += 2 * kw) {
-      const int bn = b + 2 * kw;
-      uint2 nraw0 = make_uint2(0u, 0u), nraw1 = make_uint2(0u, 0u);
-      if (bn < tot_band) {
-        nraw0 = load_key_part(a.k_idx, bidx[bn], DI);
-        nraw1 = load_key_part(a.k_idx, bidx[min(bn + 1, tot_band - 1)], DI);
-      }
-      double x0, x1;
-      if (DI == 128)
-        rescore2<128>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
-      else
-        rescore2<32>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
-      if (lane == 0) bx[b] = d2key(x0);
-      if (lane == 1 && b + 1 < tot_band) bx[b + 1] = d2key(x1);
-      raw0 = nraw0;
-      raw1 = nraw1;
+    // re-score the collected band four keys per warp call (the next four rows
+    // are loaded while the current ones are scored), rank it by (X desc,
+    // index asc), and mark the row: kept band keys -> +inf, dropped -> -inf
+    int b = warp < kw ? 4 * warp : tot_band;
+    uint2 raw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)], DI) : make_uint2(0u, 0u);
+    for (; b < tot_band; b += 4 * kw) {
+      const int bn = b + 4 * kw;
+      uint2 nraw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)], DI)
+                                : make_uint2(0u, 0u);
+      const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
+                                  : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
+      if (lane < 4 && b + lane < tot_band) bx[b + lane] = d2key(xl);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
     }
     __syncthreads();
     for (int b = threadIdx.x; b < tot_band; b += kThreads) {
@@ -628,16 +636,13 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     const int nb = static_cast<int>(nb64);
     if (flag) tile_s[j] = s;
     __syncthreads();
-    for (int jj = warp < kw ? 2 * warp : nb; jj < nb; jj += 2 * kw) {
-      const uint2 raw0 = load_key_part(a.k_idx, tile_s[jj], DI);
-      const uint2 raw1 = load_key_part(a.k_idx, tile_s[min(jj + 1, nb - 1)], DI);
-      double x0, x1;
-      if (DI == 128)
-        rescore2<128>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
-      else
-        rescore2<32>(qhi, w_lane, raw0, raw1, my_kst, HI, x0, x1);
-      if (lane == 0) tile_x[jj] = x0;
-      if (lane == 1 && jj + 1 < nb) tile_x[jj + 1] = x1;
+    for (int jj = warp < kw ? 4 * warp : nb; jj < nb; jj += 4 * kw) {
+      uint2 raw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) raw[e] = load_key_part(a.k_idx, tile_s[min(jj + e, nb - 1)], DI);
+      const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
+                                  : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
+      if (lane < 4 && jj + lane < nb) tile_x[jj + lane] = xl;
     }
     __syncthreads();
     return nb;
@@ -753,7 +758,7 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
       a.kst_extra = kKstExtraBytes;
       room = full - bytes - kKstExtraBytes;
     } else if (bytes + min_cache <= full) {
-      a.kst_warps = (kBins * 4) / (2 * 128 * 8);  // the staging fits in hist alone
+      a.kst_warps = (kBins * 4) / kKstStageBytes;  // the staging fits in hist alone
       room = full - bytes;
     } else {
       return cudaErrorInvalidConfiguration;
