@@ -436,6 +436,16 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const int qstride = a.DI + 4;
   const uint16_t* qrow = kRefine ? a.q_idx + static_cast<int64_t>(row) * a.HI * a.DI : nullptr;
 
+  // head weight of head `lane` and max ||k_idx||, loaded now and used after the
+  // select, so that their latency hides under it
+  float w_pre = 0.f;
+  unsigned long long kmax_pre = 0ull;
+  if (kRefine) {
+    const int lane0 = threadIdx.x & 31;
+    if (lane0 < a.HI) w_pre = __ldg(a.w_idx + static_cast<int64_t>(row) * a.HI + lane0);
+    kmax_pre = *reinterpret_cast<volatile unsigned long long*>(&a.ws->kmax_bits);
+  }
+
   // ---- stage the row (and the query's indexer row) with asynchronous copies
   const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
   const int n4 = n & ~3;
@@ -532,7 +542,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 #pragma unroll
     for (int u = 0; u < kHeadsPerWarp; ++u) {
       const int j = warp + u * kWarps;
-      if (j < HI) acc += fabs(static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + j])) * sqrt(ss[u]);
+      const float wj = __shfl_sync(0xffffffffu, w_pre, j & 31);
+      if (j < HI) acc += fabs(static_cast<double>(wj)) * sqrt(ss[u]);
     }
     if (lane == 0) sm.wd[warp] = acc;
   }
@@ -540,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   double A = 0.0;
   for (int w = 0; w < kWarps; ++w) A += sm.wd[w];
   A *= kNormSlack;
-  const double kmax = __longlong_as_double(static_cast<long long>(a.ws->kmax_bits));
+  const double kmax = __longlong_as_double(static_cast<long long>(kmax_pre));
   const double delta = kBoundRel * A * kmax;
   const double lo = static_cast<double>(vk) - 2.0 * delta;
   const double hi = static_cast<double>(vk) + 2.0 * delta;
@@ -578,8 +589,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     return;
   }
 
-  const double w_lane =
-      lane < HI ? static_cast<double>(a.w_idx[static_cast<int64_t>(row) * HI + lane]) : 0.0;
+  const double w_lane = lane < HI ? static_cast<double>(w_pre) : 0.0;
   uint32_t* my_kst = kst_all + warp * 512;
 
   if (tot_band <= a.bcap) {
@@ -605,15 +615,18 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < tot_band; b += kThreads) {
+    // rank of each band key by (X desc, index asc): a warp per key, its lanes
+    // counting over the band
+    for (int b = warp; b < tot_band; b += kWarps) {
       const unsigned long long xb = bx[b];
       const int sb = bidx[b];
       int rank = 0;
-      for (int o = 0; o < tot_band; ++o) {
+      for (int o = lane; o < tot_band; o += 32) {
         const unsigned long long xo = bx[o];
         rank += (xo > xb) || (xo == xb && bidx[o] < sb);
       }
-      sc[sb] = rank < r ? INFINITY : -INFINITY;
+      rank = __reduce_add_sync(0xffffffffu, rank);
+      if (lane == 0) sc[sb] = rank < r ? INFINITY : -INFINITY;
     }
     __syncthreads();
     emit_selection(
