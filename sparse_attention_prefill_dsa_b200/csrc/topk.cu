@@ -191,6 +191,23 @@ __device__ __forceinline__ void my_segment(int n, int& beg, int& end) {
   end = min(beg + len, n);
 }
 
+// Calls f(s, sc[s]) for s = beg .. end-1 in order. Eight values are loaded
+// before their calls: f writes shared memory, which the compiler must assume
+// may alias sc, so loads issued one per call would each wait for the previous
+// call's writes.
+template <class F>
+__device__ __forceinline__ void for_segment(const float* sc, int beg, int end, F f) {
+  int s = beg;
+  for (; s + 8 <= end; s += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = sc[s + u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) f(s + u, v[u]);
+  }
+  for (; s < end; ++s) f(s, sc[s]);
+}
+
 // Bucket of v in [L, U]: (v - L) * scale rounded to an integer, clamped to the
 // last bucket. Rounded float arithmetic is monotone in v, which is all the
 // select needs; ranges too narrow for a finite float scale use float64.
@@ -238,10 +255,9 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
     if (threadIdx.x == 0) sm.bc[2] = 0;
     __syncthreads();
     const Bucketer bucket(L, U);
-    for (int s = beg; s < end; ++s) {
-      const float v = sc[s];
+    for_segment(sc, beg, end, [&](int, float v) {
       if (v >= L && v <= U) atomicAdd(&hist[bucket(v)], 1);
-    }
+    });
     __syncthreads();
     int ab;
     const int bstar = find_bin_from_top<kBins>(hist, kr, &ab, sm);
@@ -249,14 +265,13 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
     above += ab;
     const int c = hist[bstar];
     float mn = INFINITY, mx = -INFINITY;
-    for (int s = beg; s < end; ++s) {
-      const float v = sc[s];
+    for_segment(sc, beg, end, [&](int, float v) {
       if (v >= L && v <= U && bucket(v) == bstar) {
         mn = fminf(mn, v);
         mx = fmaxf(mx, v);
         if (c <= kCandCap) cand[atomicAdd(&sm.bc[2], 1)] = v;
       }
-    }
+    });
     block_minmax(mn, mx, sm);  // (syncs: cand[] is complete afterwards)
     if (c <= kCandCap) {
       // rank the bucket's members: the kr-th largest value
@@ -286,32 +301,32 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
 }
 
 // Writes the selection to out[0..k): every kAbove key and the first need_ties
-// kTie keys, in ascending index order. cls(s) classifies key s.
+// kTie keys, in ascending index order. cls(v) classifies key s by v = sc[s].
 template <class Cls>
-__device__ void emit_selection(int n, int need_ties, int k, int32_t* __restrict__ out, Cls cls,
-                               Scratch& sm, WsHeader* ws, int row) {
+__device__ void emit_selection(const float* sc, int n, int need_ties, int k, int32_t* __restrict__ out,
+                               Cls cls, Scratch& sm, WsHeader* ws, int row) {
   int beg, end;
   my_segment(n, beg, end);
   unsigned int a = 0, t = 0;
-  for (int s = beg; s < end; ++s) {
-    const int c = cls(s);
+  for_segment(sc, beg, end, [&](int, float v) {
+    const int c = cls(v);
     a += c == kAbove;
     t += c == kTie;
-  }
+  });
   unsigned long long tot;
   const unsigned long long ex = block_excl_scan64(
       static_cast<unsigned long long>(a) | (static_cast<unsigned long long>(t) << 32), &tot, sm);
   int ties_before = static_cast<int>(ex >> 32);
   int pos = static_cast<int>(ex & 0xffffffffu) + min(ties_before, need_ties);
-  for (int s = beg; s < end; ++s) {
-    const int c = cls(s);
+  for_segment(sc, beg, end, [&](int s, float v) {
+    const int c = cls(v);
     bool keep = c == kAbove;
     if (c == kTie) keep = ties_before++ < need_ties;
     if (keep) {
       if (pos < k) out[pos] = s;  // never write past the row
       ++pos;
     }
-  }
+  });
   const int total =
       static_cast<int>(tot & 0xffffffffu) + min(static_cast<int>(tot >> 32), need_ties);
   if (threadIdx.x == 0 && total != k) report(ws, kDevInternal, static_cast<unsigned>(row));
@@ -496,12 +511,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   if (!kRefine) {
     emit_selection(
-        n, k - n_above, k, out,
-        [&](int s) {
-          const float v = sc[s];
-          return v > vk ? kAbove : (v == vk ? kTie : kBelow);
-        },
-        sm, a.ws, row);
+        sc, n, k - n_above, k, out,
+        [&](float v) { return v > vk ? kAbove : (v == vk ? kTie : kBelow); }, sm, a.ws, row);
     return;
   }
 
@@ -566,15 +577,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   if (threadIdx.x == 0) sm.bc[2] = 0;
   __syncthreads();
   int c_in = 0, c_band = 0;
-  for (int s = beg; s < end; ++s) {
-    const float f = sc[s];
+  for_segment(sc, beg, end, [&](int s, float f) {
     c_in += f > hi_f;
     if (f >= lo_f && f <= hi_f) {
       ++c_band;
       const int pos = atomicAdd(&sm.bc[2], 1);
       if (pos < a.bcap) bidx[pos] = s;
     }
-  }
+  });
   unsigned long long tot;
   block_excl_scan64(
       static_cast<unsigned long long>(c_in) | (static_cast<unsigned long long>(c_band) << 32),
@@ -585,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   if (r == tot_band) {  // the whole band is kept: no re-score needed
     emit_selection(
-        n, 0, k, out, [&](int s) { return sc[s] >= lo_f ? kAbove : kBelow; }, sm, a.ws, row);
+        sc, n, 0, k, out, [&](float v) { return v >= lo_f ? kAbove : kBelow; }, sm, a.ws, row);
     return;
   }
 
@@ -630,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     }
     __syncthreads();
     emit_selection(
-        n, 0, k, out, [&](int s) { return sc[s] > hi_f ? kAbove : kBelow; }, sm, a.ws, row);
+        sc, n, 0, k, out, [&](float v) { return v > hi_f ? kAbove : kBelow; }, sm, a.ws, row);
     return;
   }
 
@@ -689,9 +699,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     __syncthreads();
   }
   emit_selection(
-      n, rr, k, out,
-      [&](int s) {
-        const float v = sc[s];
+      sc, n, rr, k, out,
+      [&](float v) {
         if (isnan(v)) return kTie;
         return v > hi_f ? kAbove : kBelow;
       },
