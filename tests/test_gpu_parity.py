@@ -147,6 +147,30 @@ def test_topk_exact_mode_on_gpu_scores(dsa, oracle_lib):
     assert np.array_equal(idx.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("T", [
+    18400,   # two CTAs per SM, eight re-scoring warps, a smaller band cache
+    30000,   # one CTA per SM
+])
+def test_topk_exact_mode_launch_variants(dsa, oracle_lib, T):
+    """The top-k launch picks its shared-memory layout by context length; each
+    layout reproduces the float64 order."""
+    import torch
+
+    n_q = 6
+    d = make_dims(n_q, T - n_q, T, 32, 512, 64, 32, 128, 2048)
+    x = workloads.generate(d, 31, "normal", "uniform")
+    xd = stage(x)
+    ld = (T + 3) // 4 * 4
+    sc = torch.empty(d.n_q, ld, dtype=torch.float32, device="cuda")
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_TOPK))
+    dsa.check(dsa.dsa_index_scores(d, xd["q_idx"], xd["k_idx"], xd["w_idx"], sc, ld, ws))
+    idx = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
+    dsa.check(dsa.dsa_topk_select(d, sc, ld, xd["q_idx"], xd["k_idx"], xd["w_idx"], idx, ws))
+    dsa.check(dsa.dsa_device_status(ws))
+    ref = oracle_lib.topk_select(d, oracle_lib.index_scores(d, x["q_idx"], x["k_idx"], x["w_idx"]))
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
 def test_sparse_attn_entry_point_on_given_sets(dsa, oracle_lib):
     """dsa_sparse_attn_prefill on oracle-chosen sets, with padding and shuffled order."""
     import torch
