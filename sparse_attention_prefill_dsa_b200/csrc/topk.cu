@@ -302,17 +302,23 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
 
 // Writes the selection to out[0..k): every kAbove key and the first need_ties
 // kTie keys, in ascending index order. cls(v) classifies key s by v = sc[s].
+// a_known >= 0 is the number of kAbove keys in this thread's segment (which
+// then holds no kTie key), known to the caller; the counting pass is skipped.
 template <class Cls>
 __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int32_t* __restrict__ out,
-                               Cls cls, Scratch& sm, WsHeader* ws, int row) {
+                               Cls cls, Scratch& sm, WsHeader* ws, int row, int a_known = -1) {
   int beg, end;
   my_segment(n, beg, end);
   unsigned int a = 0, t = 0;
-  for_segment(sc, beg, end, [&](int, float v) {
-    const int c = cls(v);
-    a += c == kAbove;
-    t += c == kTie;
-  });
+  if (a_known >= 0) {
+    a = static_cast<unsigned int>(a_known);
+  } else {
+    for_segment(sc, beg, end, [&](int, float v) {
+      const int c = cls(v);
+      a += c == kAbove;
+      t += c == kTie;
+    });
+  }
   unsigned long long tot;
   const unsigned long long ex = block_excl_scan64(
       static_cast<unsigned long long>(a) | (static_cast<unsigned long long>(t) << 32), &tot, sm);
@@ -465,19 +471,36 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
   const int n4 = n & ~3;
   for (int s = threadIdx.x * 4; s < n4; s += kThreads * 4) cp_async16(sc + s, srow + s);
-  // the q row, widened to float64 once (while the copies fly); only the high
-  // words are kept
+  // the q row, widened to float64 once while the copies fly (only the high
+  // words are kept), and this warp's share of A_t = sum_j |w_j| ||q_j||
+  // (heads warp, warp + 12, ...; float64 from the widened values)
   if (kRefine) {
+    constexpr int kHeadsPerWarp = (32 + kWarps - 1) / kWarps;
     const int wpr = a.DI / 2;  // bf16 pairs per row
     const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
-    for (int e = threadIdx.x; e < a.HI * wpr; e += kThreads) {
-      const uint32_t v = __ldg(q32 + e);
-      const int j = e / wpr, c = 2 * (e - j * wpr);
-      qhi[j * qstride + c] = static_cast<uint32_t>(
-          __double2hiint(static_cast<double>(__uint_as_float(v << 16))));
-      qhi[j * qstride + c + 1] = static_cast<uint32_t>(
-          __double2hiint(static_cast<double>(__uint_as_float(v & 0xFFFF0000u))));
+    const int w0 = threadIdx.x >> 5, l0 = threadIdx.x & 31;
+    double acc = 0.0;
+#pragma unroll
+    for (int u = 0; u < kHeadsPerWarp; ++u) {
+      const int j = w0 + u * kWarps;
+      double ss = 0.0;
+      if (j < a.HI) {
+        for (int pr = l0; pr < wpr; pr += 32) {
+          const uint32_t v = __ldg(q32 + j * wpr + pr);
+          const double lo = static_cast<double>(__uint_as_float(v << 16));
+          const double hi = static_cast<double>(__uint_as_float(v & 0xFFFF0000u));
+          qhi[j * qstride + 2 * pr] = static_cast<uint32_t>(__double2hiint(lo));
+          qhi[j * qstride + 2 * pr + 1] = static_cast<uint32_t>(__double2hiint(hi));
+          ss += lo * lo;
+          ss += hi * hi;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float wj = __shfl_sync(0xffffffffu, w_pre, j & 31);
+      if (j < a.HI) acc += fabs(static_cast<double>(wj)) * sqrt(ss);
     }
+    if (l0 == 0) sm.wd[w0] = acc;
   }
   for (int s = n4 + threadIdx.x; s < n; s += kThreads) sc[s] = __ldg(srow + s);
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -530,35 +553,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   uint32_t* kst_all = reinterpret_cast<uint32_t*>(hist);
   const int kw = a.kst_warps;
 
-  // A_t = sum_j |w_j| ||q_j|| (float64 from the staged row, rounded up by a
-  // relative slack); a warp takes heads warp, warp + 8, ... together
-  {
-    constexpr int kHeadsPerWarp = (32 + kWarps - 1) / kWarps;
-    double ss[kHeadsPerWarp];
-#pragma unroll
-    for (int u = 0; u < kHeadsPerWarp; ++u) {
-      ss[u] = 0.0;
-      const int j = warp + u * kWarps;
-      if (j < HI)
-        for (int c = lane; c < DI; c += 32) {
-          const double v = __hiloint2double(static_cast<int>(qhi[j * qstride + c]), 0);
-          ss[u] += v * v;
-        }
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1)
-#pragma unroll
-      for (int u = 0; u < kHeadsPerWarp; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
-    double acc = 0.0;
-#pragma unroll
-    for (int u = 0; u < kHeadsPerWarp; ++u) {
-      const int j = warp + u * kWarps;
-      const float wj = __shfl_sync(0xffffffffu, w_pre, j & 31);
-      if (j < HI) acc += fabs(static_cast<double>(wj)) * sqrt(ss[u]);
-    }
-    if (lane == 0) sm.wd[warp] = acc;
-  }
-  __syncthreads();
+  // A_t from the warps' shares formed while the row was staged (visible
+  // since the select's block barriers), rounded up by a relative slack
   double A = 0.0;
   for (int w = 0; w < kWarps; ++w) A += sm.wd[w];
   A *= kNormSlack;
@@ -576,10 +572,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   // (any order) while they fit the cache
   if (threadIdx.x == 0) sm.bc[2] = 0;
   __syncthreads();
-  int c_in = 0, c_band = 0;
+  // (the first two band keys of the segment are noted, so that the emit can
+  // count the kept keys of the segment without a pass over it)
+  int c_in = 0, c_band = 0, bk0 = -1, bk1 = -1;
   for_segment(sc, beg, end, [&](int s, float f) {
     c_in += f > hi_f;
     if (f >= lo_f && f <= hi_f) {
+      if (c_band == 0) bk0 = s;
+      if (c_band == 1) bk1 = s;
       ++c_band;
       const int pos = atomicAdd(&sm.bc[2], 1);
       if (pos < a.bcap) bidx[pos] = s;
@@ -595,7 +595,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   if (r == tot_band) {  // the whole band is kept: no re-score needed
     emit_selection(
-        sc, n, 0, k, out, [&](float v) { return v >= lo_f ? kAbove : kBelow; }, sm, a.ws, row);
+        sc, n, 0, k, out, [&](float v) { return v >= lo_f ? kAbove : kBelow; }, sm, a.ws, row,
+        c_in + c_band);
     return;
   }
 
@@ -638,9 +639,11 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       rank = __reduce_add_sync(0xffffffffu, rank);
       if (lane == 0) sc[sb] = rank < r ? INFINITY : -INFINITY;
     }
-    __syncthreads();
+    const bool counted = __syncthreads_or(c_band > 2) == 0;
+    const int kept = c_in + (bk0 >= 0 && sc[bk0] > hi_f) + (bk1 >= 0 && sc[bk1] > hi_f);
     emit_selection(
-        sc, n, 0, k, out, [&](float v) { return v > hi_f ? kAbove : kBelow; }, sm, a.ws, row);
+        sc, n, 0, k, out, [&](float v) { return v > hi_f ? kAbove : kBelow; }, sm, a.ws, row,
+        counted ? kept : -1);
     return;
   }
 
