@@ -163,6 +163,50 @@ dsa_status dsa_prefill_layer(const dsa_dims* dims, const uint16_t* q, const uint
                              float* lse, int32_t* idx_out, void* workspace,
                              size_t workspace_bytes, void* stream);
 
+/* Device copies of the layer's tensors for dsa_prefill_layer_host, owned by
+ * the caller, each of the full size given under dsa_prefill_layer and 16-byte
+ * aligned. lse and idx may be NULL when the matching host output is NULL. */
+typedef struct {
+  uint16_t* q;
+  uint16_t* latent;
+  uint16_t* rope;
+  uint16_t* q_idx;
+  uint16_t* k_idx;
+  float* w_idx;
+  uint16_t* out;
+  float* lse;
+  int32_t* idx;
+} dsa_device_tensors;
+
+/* The whole layer on host buffers, with the host<->device copies overlapped
+ * with the compute. Query rows are independent given the cache, so the chunk
+ * is cut into n_sub consecutive sub-chunks of ceil(n_q / n_sub) rows. The call
+ * enqueues:
+ *   streams[0]: the cache (latent, rope, k_idx) into dev, then each
+ *               sub-chunk's q, q_idx and w_idx rows;
+ *   streams[1]: dsa_prefill_layer on each sub-chunk once its rows are in
+ *               (the workspace is shared by the sub-chunks, in order);
+ *   streams[2]: each sub-chunk's out (and lse, idx when given) back to the
+ *               host once its layer is done;
+ * so the copy-in of sub-chunk s+1, the layer on s and the copy-out of s-1 run
+ * together. events[0..1] are the caller's CUDA events (timing may be
+ * disabled) that the call records and waits on; streams and events are
+ * passed as cudaStream_t / cudaEvent_t cast to void*.
+ * Host inputs and outputs are the tensors of dsa_prefill_layer in host
+ * memory; page-locked memory is needed for the copies to run asynchronously.
+ * The outputs are complete once streams[2] has finished the work this call
+ * enqueued; the device status of the layer calls is read with
+ * dsa_device_status(workspace, streams[1]). Results are bit-identical to one
+ * dsa_prefill_layer call on the whole chunk.
+ * Errors: those of dsa_prefill_layer, DSA_ERR_NULL for a missing stream,
+ * event or device tensor, DSA_ERR_DIMS for n_sub < 1. */
+dsa_status dsa_prefill_layer_host(const dsa_dims* dims, const uint16_t* q, const uint16_t* latent,
+                                  const uint16_t* rope, const uint16_t* q_idx,
+                                  const uint16_t* k_idx, const float* w_idx, uint16_t* out,
+                                  float* lse, int32_t* idx_out, const dsa_device_tensors* dev,
+                                  void* workspace, size_t workspace_bytes, void* const streams[3],
+                                  void* const events[2], int32_t n_sub);
+
 /* The whole layer, as dsa_prefill_layer, for callers that cannot allocate
  * device memory: code that runs inside another engine's plugin or callback and
  * is handed only its input and output buffers, or code that must not touch the

@@ -42,7 +42,7 @@ DSA_MAX_CTX = 49152
 
 EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",
-            "dsa_status_string", "dsa_prefill_layer_noalloc")
+            "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host")
 
 
 class dsa_dims(ctypes.Structure):
@@ -59,6 +59,11 @@ class dsa_dims(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("flags", ctypes.c_uint32),
     ]
+
+
+class dsa_device_tensors(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("q", "latent", "rope", "q_idx", "k_idx", "w_idx", "out", "lse", "idx")]
 
 
 class DsaError(RuntimeError):
@@ -90,11 +95,15 @@ def library():
     lib.dsa_prefill_layer.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]
     lib.dsa_prefill_layer_noalloc.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+    lib.dsa_prefill_layer_host.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                           ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
+                                           ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int32]
     lib.dsa_device_status.argtypes = [_P, _P]
     lib.dsa_status_string.argtypes = [ctypes.c_int32]
     lib.dsa_status_string.restype = ctypes.c_char_p
     for f in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
-              "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc"):
+              "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc",
+              "dsa_prefill_layer_host"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -175,6 +184,22 @@ def dsa_prefill_layer_noalloc(dims, q, latent, rope, q_idx, k_idx, w_idx, out, l
     return library().dsa_prefill_layer_noalloc(_dims(dims), _p(q), _p(latent), _p(rope),
                                                _p(q_idx), _p(k_idx), _p(w_idx), _p(out), _p(lse),
                                                _p(idx_out), _p(device_status), _stream(stream))
+
+
+def dsa_prefill_layer_host(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out, dev,
+                           workspace, streams, events, n_sub=4, workspace_bytes=None) -> int:
+    """The layer on host buffers (q .. idx_out: page-locked host tensors or
+    addresses), copies overlapped with the compute over n_sub query
+    sub-chunks. dev maps the names of dsa_device_tensors to device tensors or
+    addresses; streams are three CUDA streams (copy in, compute, copy out),
+    events two CUDA events (torch.cuda.Event or raw cudaEvent_t addresses)."""
+    d = dsa_device_tensors(*[_p(dev.get(name)) for name, _ in dsa_device_tensors._fields_])
+    st = (_P * 3)(*[_stream(x) for x in streams])
+    ev = (_P * 2)(*[_P(x) if isinstance(x, int) else _P(x.cuda_event) for x in events])
+    return library().dsa_prefill_layer_host(_dims(dims), _p(q), _p(latent), _p(rope), _p(q_idx),
+                                            _p(k_idx), _p(w_idx), _p(out), _p(lse), _p(idx_out),
+                                            ctypes.byref(d), _p(workspace),
+                                            _nbytes(workspace, workspace_bytes), st, ev, int(n_sub))
 
 
 def dsa_device_status(workspace, stream=None) -> int:

@@ -82,6 +82,35 @@ dsa_status clear_header(void* ws, cudaStream_t st) {
   return from_cuda(cudaMemsetAsync(ws, 0, dsa::kWsHeaderBytes, st));
 }
 
+// The layer's kernels on validated arguments (the workspace header cleared
+// by the caller): scores -> exact top-k -> attention.
+dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
+                         const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
+                         const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out, void* ws,
+                         cudaStream_t st) {
+  if (d.n_q == 0) return DSA_OK;
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes);
+  const int64_t ld = layer_ld(d);
+  // The selection goes to the caller's idx_out when given, else to the
+  // workspace region after the score matrix.
+  int32_t* idx = idx_out ? idx_out : layer_idx_region(ws, d);
+  cudaError_t e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
+  if (e == cudaSuccess) e = dsa::launch_key_norm_max(d, k_idx, h, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, true, h, st));
+}
+
+cudaError_t h2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  return bytes ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st) : cudaSuccess;
+}
+
+cudaError_t d2h(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  return bytes ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, st) : cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -177,19 +206,85 @@ dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_
   if ((s = check_device()) != DSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  return enqueue_layer(*d, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out, ws, st);
+}
+
+dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
+                                  const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
+                                  const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
+                                  const dsa_device_tensors* dev, void* ws, size_t ws_bytes,
+                                  void* const streams[3], void* const events[2], int32_t n_sub) {
+  dsa_status s = check_dims(d, true, true);
+  if (s != DSA_OK) return s;
+  if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out || !dev || !streams || !events)
+    return DSA_ERR_NULL;
+  if (!events[0] || !events[1]) return DSA_ERR_NULL;
+  if (!dev->q || !dev->latent || !dev->rope || !dev->q_idx || !dev->k_idx || !dev->w_idx ||
+      !dev->out || (lse && !dev->lse) || (idx_out && !dev->idx))
+    return DSA_ERR_NULL;
+  if (!aligned16(dev->q) || !aligned16(dev->latent) || !aligned16(dev->rope) ||
+      !aligned16(dev->q_idx) || !aligned16(dev->k_idx) || !aligned16(dev->w_idx) ||
+      !aligned16(dev->out) || (dev->lse && !aligned16(dev->lse)) ||
+      (dev->idx && !aligned16(dev->idx)))
+    return DSA_ERR_ALIGN;
+  if (n_sub < 1) return DSA_ERR_DIMS;
+  if ((s = check_ws(*d, DSA_WS_LAYER, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t s_in = static_cast<cudaStream_t>(streams[0]);
+  cudaStream_t s_run = static_cast<cudaStream_t>(streams[1]);
+  cudaStream_t s_out = static_cast<cudaStream_t>(streams[2]);
+  cudaEvent_t ev_a = static_cast<cudaEvent_t>(events[0]);
+  cudaEvent_t ev_b = static_cast<cudaEvent_t>(events[1]);
+  // work already on the streams (an earlier call) ends before this call's
+  // copies overwrite the inputs its layers read and its layers overwrite the
+  // outputs its copies read
+  cudaError_t e = cudaEventRecord(ev_a, s_run);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_a, 0);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_b, s_out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_run, ev_b, 0);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  if ((s = clear_header(ws, s_run)) != DSA_OK) return s;  // once: sub-chunks keep each other's status
   if (d->n_q == 0) return DSA_OK;
-  WsHeader* h = static_cast<WsHeader*>(ws);
-  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes);
-  const int64_t ld = layer_ld(*d);
-  // The selection goes to the caller's idx_out when given, else to the
-  // workspace region after the score matrix.
-  int32_t* idx = idx_out ? idx_out : layer_idx_region(ws, *d);
-  cudaError_t e = dsa::launch_index_scores(*d, q_idx, k_idx, w_idx, scores, ld, h, st);
-  if (e == cudaSuccess) e = dsa::launch_key_norm_max(*d, k_idx, h, st);
+  const size_t T = static_cast<size_t>(d->ctx_len);
+  const size_t q_row = static_cast<size_t>(d->n_heads) * (d->d_latent + d->d_rope);
+  const size_t qi_row = static_cast<size_t>(d->n_idx_heads) * d->d_idx;
+  const size_t w_row = static_cast<size_t>(d->n_idx_heads);
+  const size_t o_row = static_cast<size_t>(d->n_heads) * d->d_latent;
+  const size_t l_row = static_cast<size_t>(d->n_heads);
+  const size_t i_row = static_cast<size_t>(d->top_k);
+  e = h2d(dev->latent, latent, T * d->d_latent * 2, s_in);
+  if (e == cudaSuccess) e = h2d(dev->rope, rope, T * d->d_rope * 2, s_in);
+  if (e == cudaSuccess) e = h2d(dev->k_idx, k_idx, T * d->d_idx * 2, s_in);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
-  e = dsa::launch_topk(*d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
-  if (e != cudaSuccess) return DSA_ERR_CUDA;
-  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, true, h, st));
+  // sub-chunks of a multiple of 4 rows keep every row offset 16-byte aligned
+  int rows = (d->n_q + n_sub - 1) / n_sub;
+  rows = (rows + 3) & ~3;
+  for (int r0 = 0; r0 < d->n_q; r0 += rows) {
+    const int nr = d->n_q - r0 < rows ? d->n_q - r0 : rows;
+    const size_t o = static_cast<size_t>(r0), n = static_cast<size_t>(nr);
+    e = h2d(dev->q + o * q_row, q + o * q_row, n * q_row * 2, s_in);
+    if (e == cudaSuccess) e = h2d(dev->q_idx + o * qi_row, q_idx + o * qi_row, n * qi_row * 2, s_in);
+    if (e == cudaSuccess) e = h2d(dev->w_idx + o * w_row, w_idx + o * w_row, n * w_row * 4, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_a, s_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_run, ev_a, 0);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    dsa_dims sub = *d;
+    sub.n_q = nr;
+    sub.q_pos0 = d->q_pos0 + r0;
+    s = enqueue_layer(sub, dev->q + o * q_row, dev->latent, dev->rope, dev->q_idx + o * qi_row,
+                      dev->k_idx, dev->w_idx + o * w_row, dev->out + o * o_row,
+                      lse ? dev->lse + o * l_row : nullptr, idx_out ? dev->idx + o * i_row : nullptr,
+                      ws, s_run);
+    if (s != DSA_OK) return s;
+    e = cudaEventRecord(ev_b, s_run);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_b, 0);
+    if (e == cudaSuccess) e = d2h(out + o * o_row, dev->out + o * o_row, n * o_row * 2, s_out);
+    if (e == cudaSuccess && lse) e = d2h(lse + o * l_row, dev->lse + o * l_row, n * l_row * 4, s_out);
+    if (e == cudaSuccess && idx_out)
+      e = d2h(idx_out + o * i_row, dev->idx + o * i_row, n * i_row * 4, s_out);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
 }
 
 dsa_status dsa_device_status(void* ws, void* stream) {

@@ -121,3 +121,34 @@ def test_valid_call_without_gpu_reports_device_error(dsa):
     d = make_dims(4, 0, 4, 4, 64, 16, 2, 32, 2)
     st = _layer(dsa, d)
     assert st in (dsa.DSA_ERR_CUDA, dsa.DSA_ERR_DEVICE)
+
+
+def test_device_tensors_struct_matches_header(dsa):
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct {\n  uint16_t* q;"):text.index("} dsa_device_tensors;")]
+    fields = re.findall(r"\*\s*([a-z_0-9]+);", body)
+    assert fields == [f for f, _ in dsa.dsa_device_tensors._fields_]
+    assert ctypes.sizeof(dsa.dsa_device_tensors) == 9 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def _host(dsa, d, dev_over=None, events=(FAKE, FAKE), n_sub=4, **over):
+    a = dict(q=FAKE, latent=FAKE, rope=FAKE, q_idx=FAKE, k_idx=FAKE, w_idx=FAKE, out=FAKE,
+             lse=None, idx_out=None, workspace=FAKE)
+    a.update(over)
+    dev = {name: FAKE for name in ("q", "latent", "rope", "q_idx", "k_idx", "w_idx", "out")}
+    dev.update(dev_over or {})
+    return dsa.dsa_prefill_layer_host(d, a["q"], a["latent"], a["rope"], a["q_idx"], a["k_idx"],
+                                      a["w_idx"], a["out"], a["lse"], a["idx_out"], dev,
+                                      a["workspace"], (0, 0, 0), events, n_sub,
+                                      workspace_bytes=dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER))
+
+
+def test_host_entry_validation_before_any_device_call(dsa):
+    d = workloads.BY_NAME["chunk2k_ctx8k"].dims
+    assert _host(dsa, d, q=None) == dsa.DSA_ERR_NULL
+    assert _host(dsa, d, dev_over={"out": None}) == dsa.DSA_ERR_NULL
+    assert _host(dsa, d, lse=FAKE) == dsa.DSA_ERR_NULL          # host lse without a device lse
+    assert _host(dsa, d, events=(FAKE, 0)) == dsa.DSA_ERR_NULL
+    assert _host(dsa, d, dev_over={"q": FAKE + 8}) == dsa.DSA_ERR_ALIGN
+    assert _host(dsa, d, n_sub=0) == dsa.DSA_ERR_DIMS
+    assert _host(dsa, d, workspace=None) == dsa.DSA_ERR_WORKSPACE

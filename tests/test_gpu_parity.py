@@ -171,6 +171,42 @@ def test_topk_exact_mode_launch_variants(dsa, oracle_lib, T):
     assert np.array_equal(idx.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("n_q,n_sub", [
+    (203, 3),   # sub-chunks of 68, 68 and 67 rows
+    (8, 8),     # rows per sub-chunk rounded up to 4: two sub-chunks
+    (64, 1),    # one sub-chunk
+])
+def test_host_entry_matches_device_entry(dsa, n_q, n_sub):
+    """dsa_prefill_layer_host (host buffers, copies overlapped with the layer
+    over query sub-chunks) gives the bits of one dsa_prefill_layer call."""
+    import torch
+
+    d, x = _reduced("chunk2k_ctx8k", n_q)
+    xd = stage(x)
+    out_ref, lse_ref, idx_ref = run_layer(dsa, d, xd)
+    pinned = {k: v.cpu().pin_memory() for k, v in xd.items()}
+    dev_t = {k: torch.empty_like(v) for k, v in xd.items()}
+    dev_t["out"] = empty_bf16(d.n_q, d.n_heads, d.d_latent)
+    dev_t["lse"] = torch.empty(d.n_q, d.n_heads, dtype=torch.float32, device="cuda")
+    dev_t["idx"] = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
+    out_h = torch.empty(d.n_q, d.n_heads, d.d_latent, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty(d.n_q, d.n_heads, dtype=torch.float32).pin_memory()
+    idx_h = torch.full((d.n_q, d.top_k), -7, dtype=torch.int32).pin_memory()
+    streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
+    events = (torch.cuda.Event(), torch.cuda.Event())
+    for ev in events:
+        ev.record()
+    ws = workspace(dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER))
+    dsa.check(dsa.dsa_prefill_layer_host(d, pinned["q"], pinned["latent"], pinned["rope"],
+                                         pinned["q_idx"], pinned["k_idx"], pinned["w_idx"], out_h,
+                                         lse_h, idx_h, dev_t, ws, streams, events, n_sub))
+    streams[2].synchronize()
+    dsa.check(dsa.dsa_device_status(ws, stream=streams[1]))
+    assert np.array_equal(host_bf16_as_f32(out_h), out_ref)
+    assert np.array_equal(lse_h.numpy(), lse_ref)
+    assert np.array_equal(idx_h.numpy(), idx_ref)
+
+
 def test_sparse_attn_entry_point_on_given_sets(dsa, oracle_lib):
     """dsa_sparse_attn_prefill on oracle-chosen sets, with padding and shuffled order."""
     import torch
