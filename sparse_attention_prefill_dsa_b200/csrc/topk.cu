@@ -479,14 +479,28 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     const int wpr = a.DI / 2;  // bf16 pairs per row
     const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
     const int w0 = threadIdx.x >> 5, l0 = threadIdx.x & 31;
+    // every bf16 pair this lane widens (at most two per head: DI <= 128) is
+    // loaded before the first is used, so the loads overlap
+    uint32_t qv[kHeadsPerWarp][2];
+#pragma unroll
+    for (int u = 0; u < kHeadsPerWarp; ++u) {
+      const int j = w0 + u * kWarps;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int pr = l0 + 32 * t;
+        qv[u][t] = (j < a.HI && pr < wpr) ? __ldg(q32 + j * wpr + pr) : 0u;
+      }
+    }
     double acc = 0.0;
 #pragma unroll
     for (int u = 0; u < kHeadsPerWarp; ++u) {
       const int j = w0 + u * kWarps;
       double ss = 0.0;
-      if (j < a.HI) {
-        for (int pr = l0; pr < wpr; pr += 32) {
-          const uint32_t v = __ldg(q32 + j * wpr + pr);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int pr = l0 + 32 * t;
+        if (j < a.HI && pr < wpr) {
+          const uint32_t v = qv[u][t];
           const double lo = static_cast<double>(__uint_as_float(v << 16));
           const double hi = static_cast<double>(__uint_as_float(v & 0xFFFF0000u));
           qhi[j * qstride + 2 * pr] = static_cast<uint32_t>(__double2hiint(lo));
