@@ -640,18 +640,29 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
     }
     __syncthreads();
-    // rank of each band key by (X desc, index asc): a warp per key, its lanes
-    // counting over the band
-    for (int b = warp; b < tot_band; b += kWarps) {
-      const unsigned long long xb = bx[b];
-      const int sb = bidx[b];
-      int rank = 0;
+    // rank of each band key by (X desc, index asc): a warp takes four keys at
+    // a time, its lanes counting over the band for all four at once
+    for (int b0 = 4 * warp; b0 < tot_band; b0 += 4 * kWarps) {
+      unsigned long long xb[4];
+      int sb[4], rank[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int b = min(b0 + e, tot_band - 1);
+        xb[e] = bx[b];
+        sb[e] = bidx[b];
+        rank[e] = 0;
+      }
       for (int o = lane; o < tot_band; o += 32) {
         const unsigned long long xo = bx[o];
-        rank += (xo > xb) || (xo == xb && bidx[o] < sb);
+        const int so = bidx[o];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rank[e] += (xo > xb[e]) || (xo == xb[e] && so < sb[e]);
       }
-      rank = __reduce_add_sync(0xffffffffu, rank);
-      if (lane == 0) sc[sb] = rank < r ? INFINITY : -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rank[e] = __reduce_add_sync(0xffffffffu, rank[e]);
+      const int my_rank = lane == 0 ? rank[0] : lane == 1 ? rank[1] : lane == 2 ? rank[2] : rank[3];
+      const int my_s = lane == 0 ? sb[0] : lane == 1 ? sb[1] : lane == 2 ? sb[2] : sb[3];
+      if (lane < 4 && b0 + lane < tot_band) sc[my_s] = my_rank < r ? INFINITY : -INFINITY;
     }
     const bool counted = __syncthreads_or(c_band > 2) == 0;
     const int kept = c_in + (bk0 >= 0 && sc[bk0] > hi_f) + (bk1 >= 0 && sc[bk1] > hi_f);
