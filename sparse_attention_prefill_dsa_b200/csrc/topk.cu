@@ -71,6 +71,7 @@ constexpr int kHist256Bytes = 256 * 4;
 // the band cache, which that path does not use
 constexpr int kSlowScratchBytes = kHist256Bytes + 4 * kThreads + 8 * kThreads;
 static_assert(kKstExtraBytes >= 0 && kKstExtraBytes % 16 == 0, "key staging");
+static_assert(kBins >= 2048, "the selection of the emit (top_k <= 2048) is staged in hist");
 
 constexpr double kDotRel = 1.0 / 32768.0;                  // 2^-15
 constexpr double kBoundRel = kDotRel + 1.0 / 131072.0;      // + 2^-17
@@ -265,14 +266,22 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
     above += ab;
     const int c = hist[bstar];
     float mn = INFINITY, mx = -INFINITY;
-    for_segment(sc, beg, end, [&](int, float v) {
-      if (v >= L && v <= U && bucket(v) == bstar) {
-        mn = fminf(mn, v);
-        mx = fmaxf(mx, v);
-        if (c <= kCandCap) cand[atomicAdd(&sm.bc[2], 1)] = v;
-      }
-    });
-    block_minmax(mn, mx, sm);  // (syncs: cand[] is complete afterwards)
+    if (c <= kCandCap) {
+      // the bucket's members into cand[] (complete after the barrier)
+      for_segment(sc, beg, end, [&](int, float v) {
+        if (v >= L && v <= U && bucket(v) == bstar) cand[atomicAdd(&sm.bc[2], 1)] = v;
+      });
+      __syncthreads();
+    } else {
+      // the bucket's value range, re-bucketed in the next round
+      for_segment(sc, beg, end, [&](int, float v) {
+        if (v >= L && v <= U && bucket(v) == bstar) {
+          mn = fminf(mn, v);
+          mx = fmaxf(mx, v);
+        }
+      });
+      block_minmax(mn, mx, sm);
+    }
     if (c <= kCandCap) {
       // rank the bucket's members: the kr-th largest value
       for (int e = threadIdx.x; e < c; e += kThreads) {
@@ -304,9 +313,12 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
 // kTie keys, in ascending index order. cls(v) classifies key s by v = sc[s].
 // a_known >= 0 is the number of kAbove keys in this thread's segment (which
 // then holds no kTie key), known to the caller; the counting pass is skipped.
+// The selection is assembled in stage[0..k) (shared memory, 16-byte aligned)
+// and then written out in coalesced pieces.
 template <class Cls>
 __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int32_t* __restrict__ out,
-                               Cls cls, Scratch& sm, WsHeader* ws, int row, int a_known = -1) {
+                               int32_t* __restrict__ stage, Cls cls, Scratch& sm, WsHeader* ws, int row,
+                               int a_known = -1) {
   int beg, end;
   my_segment(n, beg, end);
   unsigned int a = 0, t = 0;
@@ -329,13 +341,21 @@ __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int
     bool keep = c == kAbove;
     if (c == kTie) keep = ties_before++ < need_ties;
     if (keep) {
-      if (pos < k) out[pos] = s;  // never write past the row
+      if (pos < k) stage[pos] = s;  // never write past the row
       ++pos;
     }
   });
   const int total =
       static_cast<int>(tot & 0xffffffffu) + min(static_cast<int>(tot >> 32), need_ties);
   if (threadIdx.x == 0 && total != k) report(ws, kDevInternal, static_cast<unsigned>(row));
+  __syncthreads();
+  const int nw = min(total, k);
+  if ((k & 3) == 0 && nw == k) {
+    for (int i = threadIdx.x; i < k / 4; i += kThreads)
+      reinterpret_cast<int4*>(out)[i] = reinterpret_cast<const int4*>(stage)[i];
+  } else {
+    for (int i = threadIdx.x; i < nw; i += kThreads) out[i] = stage[i];
+  }
 }
 
 // Row data of a key for the float64 re-score: lane l holds dims 4l..4l+3.
@@ -548,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   if (!kRefine) {
     emit_selection(
-        sc, n, k - n_above, k, out,
+        sc, n, k - n_above, k, out, hist,
         [&](float v) { return v > vk ? kAbove : (v == vk ? kTie : kBelow); }, sm, a.ws, row);
     return;
   }
@@ -609,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   if (r == tot_band) {  // the whole band is kept: no re-score needed
     emit_selection(
-        sc, n, 0, k, out, [&](float v) { return v >= lo_f ? kAbove : kBelow; }, sm, a.ws, row,
+        sc, n, 0, k, out, hist, [&](float v) { return v >= lo_f ? kAbove : kBelow; }, sm, a.ws, row,
         c_in + c_band);
     return;
   }
@@ -667,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     const bool counted = __syncthreads_or(c_band > 2) == 0;
     const int kept = c_in + (bk0 >= 0 && sc[bk0] > hi_f) + (bk1 >= 0 && sc[bk1] > hi_f);
     emit_selection(
-        sc, n, 0, k, out, [&](float v) { return v > hi_f ? kAbove : kBelow; }, sm, a.ws, row,
+        sc, n, 0, k, out, hist, [&](float v) { return v > hi_f ? kAbove : kBelow; }, sm, a.ws, row,
         counted ? kept : -1);
     return;
   }
@@ -727,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     __syncthreads();
   }
   emit_selection(
-      sc, n, rr, k, out,
+      sc, n, rr, k, out, hist,
       [&](float v) {
         if (isnan(v)) return kTie;
         return v > hi_f ? kAbove : kBelow;
