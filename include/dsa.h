@@ -236,6 +236,23 @@ dsa_status dsa_prefill_layer_noalloc(const dsa_dims* dims, const uint16_t* q,
                                      const float* w_idx, uint16_t* out, float* lse,
                                      int32_t* idx_out, uint32_t* device_status, void* stream);
 
+/* Self-test of the failure path every kernel of the library shares: each
+ * device wait is bounded, and a wait that gives up records DSA_ERR_TIMEOUT
+ * (with the failing site) in the workspace status and makes the CTA's other
+ * waits give up too, so the CTA exits and the context stays usable. This
+ * launches one CTA of two warps that wait on barriers nothing ever signals:
+ * warp 0 with a limit of about 0.5 ms, warp 1 with the kernels' own limit
+ * (about one second), which it can only beat by following warp 0's abort.
+ * No memory outside the workspace header and `cycles` is touched.
+ *   workspace  >= dsa_workspace_size(any dims, DSA_WS_ATTN) bytes; its header
+ *              is cleared first, then receives the timeout
+ *   cycles     device int64 [2] (may be NULL): each warp's wait in SM clock
+ *              cycles
+ * Read the outcome with dsa_device_status(workspace, stream), which returns
+ * DSA_ERR_TIMEOUT. Errors: DSA_ERR_WORKSPACE, _ALIGN, _DEVICE, _CUDA. */
+dsa_status dsa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, int64_t* cycles,
+                                     void* stream);
+
 /* Synchronizes `stream`, returns the device status word of `workspace`
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_RANGE) and clears it. */
 dsa_status dsa_device_status(void* workspace, void* stream);

@@ -42,7 +42,8 @@ DSA_MAX_CTX = 49152
 
 EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",
-            "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host")
+            "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host",
+            "dsa_selftest_bounded_wait")
 
 
 class dsa_dims(ctypes.Structure):
@@ -98,12 +99,13 @@ def library():
     lib.dsa_prefill_layer_host.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
                                            ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int32]
+    lib.dsa_selftest_bounded_wait.argtypes = [_P, ctypes.c_size_t, _P, _P]
     lib.dsa_device_status.argtypes = [_P, _P]
     lib.dsa_status_string.argtypes = [ctypes.c_int32]
     lib.dsa_status_string.restype = ctypes.c_char_p
     for f in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
               "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc",
-              "dsa_prefill_layer_host"):
+              "dsa_prefill_layer_host", "dsa_selftest_bounded_wait"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -200,6 +202,13 @@ def dsa_prefill_layer_host(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse,
                                             _p(k_idx), _p(w_idx), _p(out), _p(lse), _p(idx_out),
                                             ctypes.byref(d), _p(workspace),
                                             _nbytes(workspace, workspace_bytes), st, ev, int(n_sub))
+
+
+def dsa_selftest_bounded_wait(workspace, cycles=None, workspace_bytes=None, stream=None) -> int:
+    """One CTA whose bounded waits give up (see include/dsa.h); cycles is an
+    optional device int64 tensor of 2 elements."""
+    return library().dsa_selftest_bounded_wait(_p(workspace), _nbytes(workspace, workspace_bytes),
+                                               _p(cycles), _stream(stream))
 
 
 def dsa_device_status(workspace, stream=None) -> int:

@@ -287,6 +287,17 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const ui
   return DSA_OK;
 }
 
+dsa_status dsa_selftest_bounded_wait(void* ws, size_t ws_bytes, int64_t* cycles, void* stream) {
+  if (!ws || ws_bytes < dsa::kWsHeaderBytes) return DSA_ERR_WORKSPACE;
+  if (!aligned16(ws) || (cycles && (reinterpret_cast<uintptr_t>(cycles) & 7u))) return DSA_ERR_ALIGN;
+  dsa_status s = check_device();
+  if (s != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  return from_cuda(dsa::launch_bounded_wait_selftest(static_cast<dsa::WsHeader*>(ws),
+                                                     reinterpret_cast<long long*>(cycles), st));
+}
+
 dsa_status dsa_device_status(void* ws, void* stream) {
   if (!ws) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -21,6 +21,9 @@ static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 constexpr unsigned int kDevTimeout = 1;
 constexpr unsigned int kDevRange = 2;
 constexpr unsigned int kDevInternal = 3;  // an internal consistency check failed
+// wait sites of the bounded-wait self-test (the kernels use sites below 100)
+constexpr unsigned int kSelftestSiteShort = 101;
+constexpr unsigned int kSelftestSiteLong = 102;
 constexpr size_t kWsHeaderBytes = 256;
 
 // Records the first device-side failure in the workspace header.
@@ -58,5 +61,8 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld,
 cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,
                                float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st);
+
+// The bounded-wait self-test (one CTA, two warps on mbarriers nothing signals).
+cudaError_t launch_bounded_wait_selftest(WsHeader* ws, long long* cycles, cudaStream_t st);
 
 }  // namespace dsa

@@ -53,17 +53,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 constexpr long long kWaitLimitCycles = 2000000000ll;
 
 // Waits for the phase of `bar` with the given parity. Gives up when the CTA's
-// abort flag is set or after kWaitLimitCycles; on a timeout it sets the abort
+// abort flag is set or after `limit` cycles; on a timeout it sets the abort
 // flag and records DSA_ERR_TIMEOUT (with `site`) in the workspace status.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          WsHeader* ws, unsigned site) {
+                                          WsHeader* ws, unsigned site,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         *abort_flag = 1;
         report(ws, kDevTimeout, site);
         return false;

@@ -233,6 +233,34 @@ def test_sparse_attn_entry_point_on_given_sets(dsa, oracle_lib):
 # ----------------------------------------------------------------- edge cases
 
 
+def test_bounded_wait_gives_up_cleanly(dsa, oracle_lib):
+    """The failure path the kernels share: a device wait that runs out records
+    DSA_ERR_TIMEOUT with its site, the CTA's other waits leave through the
+    abort flag instead of their own one-second limit, and the context stays
+    usable (no fault, no hang)."""
+    import time
+
+    import torch
+
+    ws = workspace(256)
+    cycles = torch.zeros(2, dtype=torch.int64, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.time()
+    dsa.check(dsa.dsa_selftest_bounded_wait(ws, cycles))
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 1.0
+    status, site = ws[:8].cpu().numpy().view(np.uint32)
+    assert status == 1 and site == 101  # timeout, at the short-limit wait
+    c = cycles.cpu().numpy()
+    assert c[0] >= 1_000_000            # warp 0 waited out its limit
+    assert 0 <= c[1] < 20_000_000       # warp 1 followed the abort, far below 2e9 cycles
+    assert dsa.dsa_device_status(ws) == dsa.DSA_ERR_TIMEOUT
+    assert dsa.dsa_device_status(ws) == dsa.DSA_OK  # read once, then cleared
+    d, x = _reduced("tiny_256q", 64)
+    out, lse, idx = run_layer(dsa, d, stage(x))
+    _compare_layer(oracle_lib, d, x, out, lse, idx)
+
+
 def test_empty_chunk_launches_nothing(dsa):
     import torch
 
