@@ -14,7 +14,8 @@ struct WsHeader {
   unsigned int status_info;   // first failing site (kernel-specific)
   unsigned long long kmax_bits;  // float64 bit pattern of max_s ||k_idx[s]||_2 (>= 0)
   unsigned int akmax_bits;       // float32 bit pattern of max_s ||[latent_s, rope_s]||_2 (>= 0)
-  unsigned char pad[236];
+  unsigned int unit_next;        // the indexer's work queue: next unit to hand out
+  unsigned char pad[232];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 

@@ -60,16 +60,19 @@ struct IdxCfg {
   static constexpr int kKSteps = DI / 16;
   static constexpr int kStepsPerChunk = kChunk / 16;
   static constexpr int kTilesPerUnit = 32;
-  static constexpr int kThreads = 320;
+  static constexpr int kEpiWarps = 8;                  // warps 2-9
+  static constexpr int kThreads = 32 * (2 + kEpiWarps);
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kM, kN, false, false);
   // shared memory carve (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffW = kOffK + kStages * kKTileBytes;        // 2 x 256 floats
   static constexpr int kOffBar = kOffW + 2 * kN * 4;
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kUnitRing = 4;                  // units handed from the producer to the others
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 2 + 1 + 2 * kUnitRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
+  static constexpr int kOffUnit = kOffMisc + 16;                     // int [kUnitRing]
+  static constexpr int kSmemBytes = kOffUnit + 4 * kUnitRing + 1024;  // + alignment slack
   static_assert(DI % 16 == 0 && kN % HI == 0 && HI <= 32 && 32 % HI == 0, "shape");
 };
 
@@ -78,20 +81,39 @@ struct IdxParams {
   float* scores;
   int64_t ld;
   int n_q, q_pos0;
-  int n_units, units_per_qb;
+  int n_units, n_qb;  // units: n_qb query blocks x (up to) kTilesPerUnit-tile slots
   WsHeader* ws;
 };
 
 template <class C>
 __device__ __forceinline__ bool unit_range(const IdxParams& p, int u, int& qb, int& kt0,
                                            int& kt1) {
-  qb = u / p.units_per_qb;
-  const int c = u - qb * p.units_per_qb;
+  // slot-major, later (longer) query blocks first: the queue hands out every
+  // block's first 32 key tiles before any block's second, so units arrive in
+  // roughly decreasing size and the CTAs finish close together
+  const int c = u / p.n_qb;
+  qb = p.n_qb - 1 - (u - c * p.n_qb);
   const int last_q = min((qb + 1) * C::kQB, p.n_q) - 1;
   const int ntiles = (p.q_pos0 + last_q) / C::kM + 1;
   kt0 = c * C::kTilesPerUnit;
   kt1 = min(kt0 + C::kTilesPerUnit, ntiles);
   return kt0 < kt1;
+}
+
+// The un-th unit of this CTA from the producer's ring (-1: the queue is
+// exhausted, or a wait gave up and *ok is false). Warp-collective; the warp
+// frees the slot once every lane has read it.
+template <class C>
+__device__ __forceinline__ int take_unit(uint64_t* unit_full, uint64_t* unit_empty, volatile int* sUnit,
+                                         uint32_t un, volatile int* abort_flag, WsHeader* ws, unsigned site,
+                                         bool& ok) {
+  const int slot = static_cast<int>(un % C::kUnitRing);
+  ok = __all_sync(0xffffffffu, mbar_wait(&unit_full[slot], (un / C::kUnitRing) & 1, abort_flag, ws, site));
+  if (!ok) return -1;
+  const int u = sUnit[slot];
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&unit_empty[slot]);
+  return u;
 }
 
 // Wait without the abort shortcut, used only to drain in-flight work.
@@ -122,8 +144,11 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
   uint64_t* w_full = acc_empty + 2;               // [2]
   uint64_t* w_empty = w_full + 2;                 // [2]
   uint64_t* mma_done = w_empty + 2;               // [1]
+  uint64_t* unit_full = mma_done + 1;             // [kUnitRing]
+  uint64_t* unit_empty = unit_full + C::kUnitRing;  // [kUnitRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* sUnit = reinterpret_cast<volatile int*>(smem + C::kOffUnit);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -136,11 +161,15 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
     mbar_init(q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);
+      mbar_init(&acc_empty[b], C::kEpiWarps);
       mbar_init(&w_full[b], 32);
-      mbar_init(&w_empty[b], 8);
+      mbar_init(&w_empty[b], C::kEpiWarps);
     }
     mbar_init(mma_done, 1);
+    for (int r = 0; r < C::kUnitRing; ++r) {
+      mbar_init(&unit_full[r], 1);
+      mbar_init(&unit_empty[r], 1 + C::kEpiWarps);  // the MMA warp and the epilogue warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -158,9 +187,32 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
     uint32_t it = 0, uq = 0;
     int q_parity_issued = -1;  // parity of the last q_full phase with copies in flight
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (uint32_t un = 0; ok; ++un) {
+      // the next non-empty unit of the queue (-1 once it is exhausted), handed
+      // to the MMA and epilogue warps through the unit ring
+      int u = -1;
+      for (;;) {
+        int v = 0;
+        if (lane == 0) v = static_cast<int>(atomicAdd(&p.ws->unit_next, 1u));
+        v = __shfl_sync(0xffffffffu, v, 0);
+        if (v >= p.n_units) break;
+        int qb_, kt0_, kt1_;
+        if (unit_range<C>(p, v, qb_, kt0_, kt1_)) {
+          u = v;
+          break;
+        }
+      }
+      const int slot = static_cast<int>(un % C::kUnitRing);
+      ok = __all_sync(0xffffffffu, mbar_wait(&unit_empty[slot], ((un / C::kUnitRing) & 1) ^ 1, abort_flag,
+                                             p.ws, 9));
+      if (!ok) break;
+      if (lane == 0) {
+        sUnit[slot] = u;
+        mbar_arrive(&unit_full[slot]);
+      }
+      if (u < 0) break;
       int qb, kt0, kt1;
-      if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+      unit_range<C>(p, u, qb, kt0, kt1);
       // head weights of the block -> sW[uq & 1] (all 32 lanes write and arrive)
       const int wb = uq & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&w_empty[wb], ((uq >> 1) & 1) ^ 1, abort_flag, p.ws, 1));
@@ -211,9 +263,11 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
     bool ok = true;
     const uint64_t dk0 = smem_desc(smem_u32(sK), 16, C::kSbo, C::kSwzCode);
     const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, C::kSbo, C::kSwzCode);
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (uint32_t un = 0; ok; ++un) {
+      const int u = take_unit<C>(unit_full, unit_empty, sUnit, un, abort_flag, p.ws, 10, ok);
+      if (u < 0) break;
       int qb, kt0, kt1;
-      if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+      unit_range<C>(p, u, qb, kt0, kt1);
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full, uq & 1, abort_flag, p.ws, 4)))) break;
       for (int kt = kt0; kt < kt1; ++kt, ++it) {
         const int st = it % C::kStages, buf = it & 1;
@@ -252,9 +306,11 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     uint32_t it = 0, uq = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (uint32_t un = 0; ok; ++un) {
+      const int u = take_unit<C>(unit_full, unit_empty, sUnit, un, abort_flag, p.ws, 11, ok);
+      if (u < 0) break;
       int qb, kt0, kt1;
-      if (!unit_range<C>(p, u, qb, kt0, kt1)) continue;
+      unit_range<C>(p, u, qb, kt0, kt1);
       const int wb = uq & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&w_full[wb], (uq >> 1) & 1, abort_flag, p.ws, 7));
       if (!ok) break;
@@ -343,9 +399,12 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_i
   p.q_pos0 = d.q_pos0;
   p.ws = ws;
   const int max_tiles = (d.q_pos0 + d.n_q - 1) / C::kM + 1;
-  p.units_per_qb = (max_tiles + C::kTilesPerUnit - 1) / C::kTilesPerUnit;
-  const int n_qb = (d.n_q + C::kQB - 1) / C::kQB;
-  p.n_units = n_qb * p.units_per_qb;
+  const int slots = (max_tiles + C::kTilesPerUnit - 1) / C::kTilesPerUnit;
+  p.n_qb = (d.n_q + C::kQB - 1) / C::kQB;
+  p.n_units = p.n_qb * slots;
+  // the work queue starts at unit 0 on every launch
+  cudaError_t e0 = cudaMemsetAsync(&ws->unit_next, 0, sizeof(ws->unit_next), st);
+  if (e0 != cudaSuccess) return e0;
   const int grid = p.n_units < num_sms() ? p.n_units : num_sms();
   // The CTA owns all 512 TMEM columns of its SM: ask for enough shared memory
   // that a second CTA can never be resident beside it.
