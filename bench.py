@@ -47,7 +47,7 @@ PROFILED_DRAM_BYTES_PER_QUERY = {
 }
 
 KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
-E2E_SUB_CHUNKS = (4, 8, 16, 32)  # query sub-chunk counts tried for the host-buffer call (copies overlap the layer)
+E2E_SUB_CHUNKS = (8, 16, 32, 64)  # query sub-chunk counts tried for the host-buffer call (copies overlap the layer)
 
 
 def load_peaks():
