@@ -14,8 +14,11 @@ host->device copies of the inputs and the device->host copy of the output
 inside the timed region. ``--impl reference`` times the float64 CPU oracle on
 a bounded sample of the same workload instead.
 
-Multi-GPU (torchrun): every rank runs its own chunk of the same shape (weak
-scaling, no data-path collective); the step time is the max over ranks.
+Multi-GPU (torchrun): by default every rank runs its own chunk of the same
+shape (weak scaling, no data-path collective); with ``--split query`` one chunk
+is split by queries over the ranks (strong scaling: the chunk's new cache rows
+and the outputs are all-gathered over NCCL inside each step). The step time is
+the max over ranks.
 """
 from __future__ import annotations
 
@@ -38,13 +41,11 @@ import workloads  # noqa: E402
 SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + write) per query of one kernel launch, from the ncu capture
-# named beside each entry; traffic scales with the query count (q rows, outputs,
-# index rows), so a launch's traffic is this figure times n_q. An entry is
-# removed whenever its kernel changes after the capture.
-PROFILED_DRAM_BYTES_PER_QUERY = {
-    "sparse_attn": (141.63e6 / 2048, "profiles/sparse_attn_tc_chunk2k_ctx8k.md"),
-}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
+# kernel inside the layer on a workload, from one ncu capture of that launch
+# (bench.py --layer-only on the same workload). An entry is removed whenever
+# its kernel changes after the capture.
+PROFILED_DRAM_BYTES_PER_LAUNCH: dict = {}
 
 KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
 E2E_SUB_CHUNKS = (8, 16, 32, 64)  # query sub-chunk counts tried for the host-buffer call (copies overlap the layer)
@@ -197,6 +198,46 @@ class ClockSampler:
 # ------------------------------------------------------------ our GPU path
 
 
+def kernel_rates(d, per_kernel_ms, peaks):
+    """Useful rate and roofline fraction of each entry point's kernels.
+
+    The indexer and the attention are contractions (useful FLOP / time against
+    the bf16 peak); the top-k reads each causal score once and writes the
+    selection (algorithmic bytes / time against the HBM copy bandwidth)."""
+    fl = workloads.useful_flops(d)
+    t = d.q_pos0 + np.arange(d.n_q, dtype=np.int64)
+    topk_bytes = float(((t + 1) * 4).sum() + d.n_q * d.top_k * 4)
+    out = {}
+    for name, ms in per_kernel_ms.items():
+        if name == "topk_select":
+            ach = topk_bytes / (ms / 1e3) / 1e9
+            out[name] = {"ms": ms, "bound": "hbm", "achieved": ach, "unit": "GB/s",
+                         "algorithmic": topk_bytes, "frac": ach / peaks["hbm_gbs"]}
+        else:
+            f = fl["indexer"] if name == "index_scores" else fl["attention"]
+            ach = f / (ms / 1e3) / 1e12
+            out[name] = {"ms": ms, "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                         "algorithmic": float(f), "frac": ach / peaks["bf16_tflops"]}
+    return out
+
+
+def time_steps(step, flush, steps, stream, flushed=True):
+    """CUDA-event time of each of `steps` calls of step() on `stream`; with
+    flushed=True the L2 is overwritten (untimed) before each step."""
+    import torch
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for s in range(steps):
+        if flushed:
+            flush.zero_()
+        starts[s].record(stream)
+        step()
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in zip(starts, ends)]
+
+
 def run_ours(args):
     import torch
 
@@ -243,30 +284,40 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # ---- timed region: K steps of the layer, L2 flushed (untimed) between steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clocks:
-        for s in range(args.steps):
-            flush.zero_()
-            starts[s].record(stream)
-            layer()
-            ends[s].record(stream)
-        torch.cuda.synchronize()
+        step_ms = time_steps(layer, flush, args.steps, stream)
     barrier(world)
     dsa.check(dsa.dsa_device_status(ws_layer, stream=stream))
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     value = whole_job_rate(world, d.n_q, ms_per_step)
+    fl = workloads.useful_flops(d)
+    peaks, peaks_src = load_peaks()
+    tflops = fl["total"] / (ms_per_step / 1e3) / 1e12
+    if args.layer_only:  # the layer alone (for profiler captures): no other legs
+        if rank == 0:
+            print(json.dumps({"metric": "DSA prefill queries/s per layer", "value": value,
+                              "unit": "queries/s", "ms_per_step": ms_per_step,
+                              "workload": wl.name, "tflops": tflops,
+                              "clocks": clocks.summary()}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    # ---- the same layer with a warm L2 (no flush between steps)
+    warm_ms = time_steps(layer, flush, args.steps, stream, flushed=False)
+    warm_ms_per_step = max_over_ranks(statistics.median(warm_ms), world)
 
     # ---- per-kernel durations, same inputs and launch configuration
     ld = (d.ctx_len + 127) // 128 * 128
     scores = ws_layer[256:256 + d.n_q * ld * 4].view(torch.float32).view(d.n_q, ld)
     ws_small = torch.empty(256, dtype=torch.uint8, device="cuda")
     names = ("index_scores", "topk_select", "sparse_attn")
-    ev = {n: [] for n in names}
+    ev = []
     for s in range(args.steps):
         flush.zero_()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -280,13 +331,11 @@ def run_ours(args):
         dsa.check(dsa.dsa_sparse_attn_prefill(d, xd["q"], xd["latent"], xd["rope"], idx, out,
                                               lse, ws_small, stream=stream))
         e[3].record(stream)
-        ev["index_scores"].append(e)
+        ev.append(e)
     torch.cuda.synchronize()
-    per_kernel = {n: 0.0 for n in names}
-    for e in ev["index_scores"]:
-        per_kernel["index_scores"] += e[0].elapsed_time(e[1]) / args.steps
-        per_kernel["topk_select"] += e[1].elapsed_time(e[2]) / args.steps
-        per_kernel["sparse_attn"] += e[2].elapsed_time(e[3]) / args.steps
+    per_kernel = {n: statistics.median(e[j].elapsed_time(e[j + 1]) for e in ev)
+                  for j, n in enumerate(names)}
+    rates = kernel_rates(d, per_kernel, peaks)
 
     # ---- end to end through the library's host-buffer call: every step copies
     # all inputs in from page-locked host memory and the output back, the
@@ -336,27 +385,19 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     barrier(world)
 
-    fl = workloads.useful_flops(d)
-    peaks, peaks_src = load_peaks()
-    tflops = fl["total"] * world / (ms_per_step / 1e3) / 1e12 / world
+    # the dominant kernel's roofline, with its DRAM traffic when a capture of
+    # the current kernel on this workload exists
     dom_name = max(per_kernel, key=per_kernel.get)
-    dom_flops = {"index_scores": fl["indexer"], "sparse_attn": fl["attention"]}
-    if dom_name in dom_flops:
-        ach = dom_flops[dom_name] / (per_kernel[dom_name] / 1e3) / 1e12
-        prof = PROFILED_DRAM_BYTES_PER_QUERY.get(dom_name)
-        roof = {"kernel": dom_name, "bound": "tensor", "achieved": ach,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"],
-                "traffic": prof[0] * d.n_q if prof else None,
-                "traffic_source": (f"{prof[1]} (DRAM bytes per query x n_q)" if prof else None),
-                "peak_source": f"{peaks_src} bf16 burst (kernel timed alone)"}
-    else:  # top-k reads the score rows once
-        t = d.q_pos0 + np.arange(d.n_q)
-        nbytes = float(((t + 1) * 4).sum() + d.n_q * d.top_k * 4)
-        ach = nbytes / (per_kernel[dom_name] / 1e3) / 1e9
-        roof = {"kernel": dom_name, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
-                "peak_source": f"{peaks_src} copy bandwidth"}
+    r = rates[dom_name]
+    prof = PROFILED_DRAM_BYTES_PER_LAUNCH.get((dom_name, wl.name))
+    roof = {"kernel": dom_name, "bound": r["bound"], "achieved": r["achieved"],
+            "peak": peaks["bf16_tflops"] if r["bound"] == "tensor" else peaks["hbm_gbs"],
+            "unit": r["unit"], "frac": r["frac"],
+            "traffic": prof if prof else None,
+            "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch of "
+                               "this kernel inside the layer on this workload" if prof else None),
+            "peak_source": (f"{peaks_src} bf16 burst (kernel timed alone)" if r["bound"] == "tensor"
+                            else f"{peaks_src} copy bandwidth")}
 
     result = {
         "metric": "DSA prefill queries/s per layer",
@@ -380,7 +421,11 @@ def run_ours(args):
         "pct_of_measured_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
         "pct_of_spec_bf16_peak": 100.0 * tflops / SPEC_BF16_TFLOPS,
         "useful_flop_per_step": fl["total"],
+        "ms_per_step_median": max_over_ranks(statistics.median(step_ms), world),
+        "warm_l2": {"ms_per_step_median": warm_ms_per_step,
+                    "value": whole_job_rate(world, d.n_q, warm_ms_per_step)},
         "per_kernel_ms": per_kernel,
+        "per_kernel": rates,
         "e2e": {"value": whole_job_rate(world, d.n_q, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "call": "dsa_prefill_layer_host", "sub_chunks": n_best,
@@ -394,6 +439,123 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
 
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_split(args):
+    """One chunk split by queries over the ranks (strong scaling): each step
+    gathers the chunk's new cache rows, runs the layer on this rank's query
+    range (dsa_partition_queries) and gathers the outputs, all over NCCL."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_prefill_dsa_b200 as dsa
+    from sparse_attention_prefill_dsa_b200 import multi_gpu
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dsa.library()
+    wl = workloads.BY_NAME[args.workload]
+    d = wl.dims
+    w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
+    x = workloads.generate(d, wl.seed, wl.kind, w_mode)  # one chunk, the same on every rank
+    stream = torch.cuda.current_stream()
+
+    def to_dev(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
+            else torch.from_numpy(a)
+        return t.cuda()
+
+    cache = {k: to_dev(x[k]) for k in ("latent", "rope", "k_idx")}
+    chunk = {k: to_dev(x[k]) for k in ("q", "q_idx", "w_idx")}
+    outputs = {"out": torch.empty(d.n_q, d.n_heads, d.d_latent, dtype=torch.bfloat16,
+                                  device="cuda")}
+    ranges = multi_gpu.query_ranges(d, world)
+    s0, e0 = ranges[rank]
+    ws = torch.empty(dsa.dsa_workspace_size(multi_gpu.sub_dims(d, s0, e0), dsa.DSA_WS_LAYER),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def layer_fn(sd, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx):
+        dsa.check(dsa.dsa_prefill_layer(sd, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx,
+                                        ws, stream=stream))
+
+    def step():
+        multi_gpu.prefill_layer_sharded(d, rank, world, cache, chunk, outputs, layer_fn)
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    dsa.check(dsa.dsa_device_status(ws, stream=stream))
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        step_ms = time_steps(step, flush, args.steps, stream)
+    barrier(world)
+    dsa.check(dsa.dsa_device_status(ws, stream=stream))
+    ms_per_step = max_over_ranks(sum(step_ms), world) / args.steps
+    value = d.n_q / (ms_per_step / 1e3)
+
+    # end to end: this rank's inputs (its chunk rows and the prefix cache) in
+    # from page-locked host memory, the gathered output back out, every step
+    pinned = {k: (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
+                  if v.dtype == np.uint16 else torch.from_numpy(v)).pin_memory()
+              for k, v in x.items()}
+    out_host = torch.empty(outputs["out"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = 0
+    for k in ("latent", "rope", "k_idx"):
+        h2d += (d.q_pos0 + e0 - s0) * pinned[k][0].numel() * pinned[k].element_size()
+    for k in ("q", "q_idx", "w_idx"):
+        h2d += (e0 - s0) * pinned[k][0].numel() * pinned[k].element_size()
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e():
+        for k in ("latent", "rope", "k_idx"):
+            cache[k][: d.q_pos0].copy_(pinned[k][: d.q_pos0], non_blocking=True)
+            cache[k][d.q_pos0 + s0: d.q_pos0 + e0].copy_(
+                pinned[k][d.q_pos0 + s0: d.q_pos0 + e0], non_blocking=True)
+        for k in ("q", "q_idx", "w_idx"):
+            chunk[k][s0:e0].copy_(pinned[k][s0:e0], non_blocking=True)
+        step()
+        out_host.copy_(outputs["out"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
+    fl = workloads.useful_flops(d)
+    peaks, _ = load_peaks()
+    tflops = fl["total"] / (ms_per_step / 1e3) / 1e12
+    result = {
+        "metric": "DSA prefill queries/s per layer", "value": value, "unit": "queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "about": wl.about, "n_q": d.n_q, "ctx_len": d.ctx_len,
+                   "top_k": d.top_k, "parallelism": f"query split over {world} ranks "
+                   "(cache rows and outputs all-gathered over NCCL)",
+                   "ranges": ranges, "l2": "flushed: 256 MB write between timed steps"},
+        "tflops": tflops, "pct_of_measured_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "e2e": {"value": d.n_q / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": KERNELS_PER_LAYER * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
@@ -476,11 +638,18 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="query rows of the bounded CPU-oracle sample (0: about 12 s of work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", default="chunks", choices=("chunks", "query"),
+                    help="chunks: every rank runs its own chunk (weak scaling, default); "
+                         "query: one chunk split by queries over the ranks (strong scaling)")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="time the layer alone and print a short line (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.split == "query":
+        run_split(args)
     else:
         run_ours(args)
 

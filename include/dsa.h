@@ -142,11 +142,12 @@ dsa_status dsa_topk_select(const dsa_dims* dims, const float* scores, int64_t ld
  *   q      bf16  [n_q, n_heads, d_latent + d_rope]
  *   latent bf16  [ctx_len, d_latent]
  *   rope   bf16  [ctx_len, d_rope]
- *   idx    int32 [n_q, top_k], every valid entry in 0..ctx_len-1
+ *   idx    int32 [n_q, top_k], every valid entry of row i in 0..t, t = q_pos0 + i
+ *          (the keys a causal query may see)
  *   out    bf16  [n_q, n_heads, d_latent] (output)
  *   lse    f32   [n_q, n_heads] (output) or NULL
- * Out-of-range indices are not read; they set DSA_ERR_RANGE in the workspace
- * status and that key is skipped.
+ * An index past t (a future token, or past the cache) is not read; it sets
+ * DSA_ERR_RANGE in the workspace status and that key is skipped.
  * Errors: DSA_ERR_NULL, _ALIGN, _DIMS, _CAUSAL, _WORKSPACE, _DEVICE, _CUDA. */
 dsa_status dsa_sparse_attn_prefill(const dsa_dims* dims, const uint16_t* q,
                                    const uint16_t* latent, const uint16_t* rope,
@@ -216,11 +217,16 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* dims, const uint16_t* q, const
  * The scratch (score rows, selections, status word) lives in a static device
  * array of DSA_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads the
  * library holds until the process exits. The call allocates nothing:
- *  - chunks whose dsa_workspace_size(dims, DSA_WS_LAYER) exceeds
- *    DSA_NOALLOC_SCRATCH_BYTES return DSA_ERR_SCRATCH_LIMIT (e.g. 1,024 queries
- *    fit up to a ~6K context at top_k 2048; split larger chunks);
+ *  - chunks whose dsa_workspace_size(dims, DSA_WS_LAYER), i.e.
+ *        256 + n_q * (round_up(ctx_len, 128) + top_k) * 4 bytes,
+ *    exceeds DSA_NOALLOC_SCRATCH_BYTES return DSA_ERR_SCRATCH_LIMIT (e.g.
+ *    1,024 queries at top_k 2048 fit up to a 6,016-token context; split larger
+ *    chunks). The selection region counts even when idx_out is given;
  *  - the first call on each device looks up the array's device address with
- *    that device current; make that first call before any stream capture;
+ *    that device current, and so does the first call after the device's
+ *    context was destroyed and created anew (cudaDeviceReset, or the primary
+ *    context released and retained again); make those calls before any stream
+ *    capture;
  *  - all calls on a device share the array, and it keeps the last call's
  *    contents: calls that overlap on the GPU (other streams, other threads)
  *    race on it. Each call clears the status word and scalars it relies on.
@@ -235,6 +241,22 @@ dsa_status dsa_prefill_layer_noalloc(const dsa_dims* dims, const uint16_t* q,
                                      const uint16_t* q_idx, const uint16_t* k_idx,
                                      const float* w_idx, uint16_t* out, float* lse,
                                      int32_t* idx_out, uint32_t* device_status, void* stream);
+
+/* Multi-GPU prefill of one chunk: splits its queries into n_parts contiguous
+ * ranges, one per rank, with nearly equal useful work. Row i (position t)
+ * costs (t+1) * 2 * n_idx_heads * d_idx multiply-adds in the indexer and
+ * min(top_k, t+1) * 2 * n_heads * (2 d_latent + d_rope) in the attention, so
+ * later rows are dearer and equal row counts would overload the last rank.
+ * Part p takes rows starts[p] .. starts[p+1]-1; rank p then calls
+ * dsa_prefill_layer with n_q = starts[p+1] - starts[p], q_pos0 advanced by
+ * starts[p] and its row slices of q, q_idx, w_idx, out, lse and idx, against
+ * the whole cache. Boundaries are multiples of the smallest row count that
+ * keeps every per-row tensor offset 16-byte aligned (1 for the 32-head shapes
+ * at a top_k that is a multiple of 4, at most 8); a part may be empty.
+ *   starts  host int32 [n_parts + 1] (output), starts[0] = 0, starts[n_parts] = n_q
+ * Host arithmetic only: no device is touched and nothing is allocated on one.
+ * Errors: DSA_ERR_NULL, _DIMS (n_parts < 1 or a nonpositive size), _CAUSAL. */
+dsa_status dsa_partition_queries(const dsa_dims* dims, int32_t n_parts, int32_t* starts);
 
 /* Self-test of the failure path every kernel of the library shares: each
  * device wait is bounded, and a wait that gives up records DSA_ERR_TIMEOUT

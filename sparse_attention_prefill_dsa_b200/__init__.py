@@ -8,6 +8,11 @@ RuntimeError when libdsa.so has not been built.
 
 Tensors may be given as torch tensors (their data_ptr() is passed) or as raw
 integer device addresses. ``stream`` defaults to torch's current CUDA stream.
+
+DSA_LIBRARY=check in the environment loads libdsa_check.so instead: the same
+kernels built with bounds checks that report a bad index in the workspace
+status (DSA_ERR_CUDA from dsa_device_status, site 1000 + n in the header)
+rather than making the access.
 """
 from __future__ import annotations
 
@@ -15,7 +20,8 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libdsa.so")
+LIB_PATH = os.path.join(_PKG, "libdsa_check.so" if os.environ.get("DSA_LIBRARY") == "check"
+                        else "libdsa.so")
 
 _lib = None
 
@@ -43,7 +49,7 @@ DSA_MAX_CTX = 49152
 EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",
             "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host",
-            "dsa_selftest_bounded_wait")
+            "dsa_selftest_bounded_wait", "dsa_partition_queries")
 
 
 class dsa_dims(ctypes.Structure):
@@ -100,12 +106,13 @@ def library():
                                            ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
                                            ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int32]
     lib.dsa_selftest_bounded_wait.argtypes = [_P, ctypes.c_size_t, _P, _P]
+    lib.dsa_partition_queries.argtypes = [_DP, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     lib.dsa_device_status.argtypes = [_P, _P]
     lib.dsa_status_string.argtypes = [ctypes.c_int32]
     lib.dsa_status_string.restype = ctypes.c_char_p
     for f in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
               "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc",
-              "dsa_prefill_layer_host", "dsa_selftest_bounded_wait"):
+              "dsa_prefill_layer_host", "dsa_selftest_bounded_wait", "dsa_partition_queries"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -224,3 +231,14 @@ def check(status: int) -> None:
     if status != DSA_OK:
         raise DsaError(status)
 
+
+
+def dsa_partition_queries(dims, n_parts: int, starts=None):
+    """Query ranges of one chunk over n_parts ranks (see include/dsa.h).
+    Returns (status, starts) with starts a list of n_parts + 1 row offsets."""
+    arr = (ctypes.c_int32 * (int(n_parts) + 1))() if n_parts >= 1 else (ctypes.c_int32 * 1)()
+    st = library().dsa_partition_queries(_dims(dims), int(n_parts), arr)
+    out = list(arr)
+    if starts is not None:
+        starts[:] = out
+    return st, out

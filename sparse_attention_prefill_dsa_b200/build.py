@@ -1,6 +1,9 @@
-"""Builds libdsa.so (the C-ABI library) in-tree with nvcc for sm_100a.
+"""Builds libdsa.so (the C-ABI library) in-tree with nvcc for sm_100a, and its
+checking variant libdsa_check.so (the same sources with -DDSA_CHECK=1: every
+dynamically indexed buffer access is bounds-checked and a bad index is
+reported in the workspace status instead of being made).
 
-Usage: python -m sparse_attention_prefill_dsa_b200.build [--verbose]
+Usage: python -m sparse_attention_prefill_dsa_b200.build [--verbose] [--check]
 """
 from __future__ import annotations
 
@@ -16,6 +19,11 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(PKG, "libdsa.so")
 BUILD = os.path.join(PKG, "_build")
+VARIANTS = {  # name -> (library, object folder, extra nvcc flags)
+    "release": (OUT, BUILD, []),
+    "check": (os.path.join(PKG, "libdsa_check.so"), os.path.join(PKG, "_build_check"),
+              ["-DDSA_CHECK=1"]),
+}
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
@@ -38,17 +46,18 @@ def _deps() -> list[str]:
     return files + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(OUT):
+def build(force: bool = False, verbose: bool = False, variant: str = "release") -> str:
+    out, build_dir, vflags = VARIANTS[variant]
+    if not force and os.path.exists(out):
         newest = max(os.path.getmtime(p) for p in _deps())
-        if os.path.getmtime(OUT) >= newest:
-            return OUT
+        if os.path.getmtime(out) >= newest:
+            return out
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if verbose else []
+    os.makedirs(build_dir, exist_ok=True)
+    extra = (["-Xptxas", "-v"] if verbose else []) + vflags
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -60,12 +69,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
-    tmp = OUT + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results]]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    print(build(force=True, verbose="--verbose" in sys.argv,
+                variant="check" if "--check" in sys.argv else "release"))

@@ -394,11 +394,12 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
 #pragma unroll
         for (int e = 0; e < R; ++e) {
           int row = cur[e];
-          if (row >= p.ctx_len) {
+          if (row > p.q_pos0 + i) {  // past the query's own position (t < ctx_len)
             report(p.ws, kDevRange, static_cast<unsigned>(i));
             row = -1;
           }
           if (row < 0) row = 0;  // masked key: any valid row, weight zero
+          if (!DSA_IN_BOUNDS(p.ws, row, p.ctx_len, 13)) row = 0;
           lsrc[e] = p.latent + static_cast<int64_t>(row) * DC + part * 8;
           rsrc[e] = p.rope + static_cast<int64_t>(row) * DR + part * 8;
         }
@@ -406,7 +407,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         if (!ok) break;
         if (part < DR / 8) {
 #pragma unroll
-          for (int e = 0; e < R; ++e) cp_async_16(sRope + doff[e], rsrc[e]);
+          for (int e = 0; e < R; ++e)
+            if (DSA_IN_BOUNDS(p.ws, doff[e] + 16, C::kChunkBytes + 1, 10)) cp_async_16(sRope + doff[e], rsrc[e]);
         }
         cp_async_arrive_noinc(rope_full);
 #pragma unroll
@@ -423,7 +425,9 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             if (c < C::NL) {
 #pragma unroll
               for (int e = 0; e < R; ++e)
-                cp_async_16(dst + half * C::kChunkBytes + doff[e], lsrc[e] + c * 64);
+                if (DSA_IN_BOUNDS(p.ws, pi * C::kPairBytes + half * C::kChunkBytes + doff[e] + 16,
+                                  C::kPairs * C::kPairBytes + 1, 14))
+                  cp_async_16(dst + half * C::kChunkBytes + doff[e], lsrc[e] + c * 64);
               cp_async_arrive_noinc(&pair_full[2 * pi + half]);
             }
           }
@@ -567,7 +571,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           sNorm[sw * 32 + lane] = qn2;
         }
         const bool issue_q = j == nt - 1 && q_loader && next_q;
-        const bool valid = row >= 0 && row < p.ctx_len;
+        const bool valid = row >= 0 && row <= p.q_pos0 + i;
         if (!fixed_m) {
           // per-head maximum of this tile over all 128 keys (log2 units)
           float red[HH];
@@ -662,6 +666,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[0], pv[1]);
             w4[e2] = *reinterpret_cast<const uint32_t*>(&b2);
           }
+          if (DSA_IN_BOUNDS(p.ws, r * C::kPRowBytes + ((c ^ swz) << 4) + 16, C::kPBytes + 1, 11))
           *reinterpret_cast<uint4*>(prow + ((c ^ swz) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         fence_proxy_async_smem();
@@ -698,7 +703,10 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           uint16_t* orow = p.out + (static_cast<int64_t>(i) * H + hh * HH) * DC + d;
 #pragma unroll
           for (int h = 0; h < HH; ++h)
-            if (hh * HH + h < H) orow[h * DC] = f32_to_bf16_rne(o[h] * inv[h]);
+            if (hh * HH + h < H &&
+                DSA_IN_BOUNDS(p.ws, (static_cast<int64_t>(i) * H + hh * HH + h) * DC + d,
+                              static_cast<int64_t>(p.n_q) * H * DC, 12))
+              orow[h * DC] = f32_to_bf16_rne(o[h] * inv[h]);
         }
       }
       tc_fence_before();
@@ -778,12 +786,6 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
   if (!make_tmap_bf16_2d(&tm_q, q, DC + DR, static_cast<uint64_t>(d.n_q) * H, 64, H,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  {
-    const int threads = 256;
-    int blocks = (d.ctx_len * 32 + threads - 1) / threads;
-    if (blocks > num_sms() * 8) blocks = num_sms() * 8;
-    attn_key_norm_max_kernel<DC, DR><<<blocks, threads, 0, st>>>(latent, rope, d.ctx_len, ws);
-  }
   const int grid = d.n_q < num_sms() ? d.n_q : num_sms();
   const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc<H, DC, DR>,
@@ -793,7 +795,24 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
   return cudaGetLastError();
 }
 
+template <int DC, int DR>
+cudaError_t launch_norm(const dsa_dims& d, const uint16_t* latent, const uint16_t* rope, WsHeader* ws,
+                        cudaStream_t st) {
+  const int threads = 256;
+  int blocks = (d.ctx_len * 32 + threads - 1) / threads;
+  if (blocks > num_sms() * 8) blocks = num_sms() * 8;
+  attn_key_norm_max_kernel<DC, DR><<<blocks, threads, 0, st>>>(latent, rope, d.ctx_len, ws);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_attn_key_norm_max(const dsa_dims& d, const uint16_t* latent, const uint16_t* rope,
+                                     WsHeader* ws, cudaStream_t st) {
+  if (d.d_latent == 512 && d.d_rope == 64) return launch_norm<512, 64>(d, latent, rope, ws, st);
+  if (d.d_latent == 64 && d.d_rope == 16) return launch_norm<64, 16>(d, latent, rope, ws, st);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,

@@ -13,12 +13,13 @@
 
 using dsa::WsHeader;
 
+namespace dsa {
 namespace {
-
 constexpr int kMaxDevices = 64;
 int g_device_ok[kMaxDevices];  // 0 unknown, 1 sm_100, -1 other
+}  // namespace
 
-dsa_status check_device() {
+dsa_status check_current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_DEVICE;
@@ -31,6 +32,12 @@ dsa_status check_device() {
   }
   return g_device_ok[dev] == 1 ? DSA_OK : DSA_ERR_DEVICE;
 }
+
+}  // namespace dsa
+
+namespace {
+
+dsa_status check_device() { return dsa::check_current_device(); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -83,11 +90,15 @@ dsa_status clear_header(void* ws, cudaStream_t st) {
 }
 
 // The layer's kernels on validated arguments (the workspace header cleared
-// by the caller): scores -> exact top-k -> attention.
+// by the caller): scores -> exact top-k -> attention. The two key-norm passes
+// (max ||k_idx[s]|| for the top-k band, max ||[latent_s, rope_s]|| for the
+// attention's score bound) depend only on the cache, so a caller that runs
+// several sub-chunks against one cache and one header computes them once
+// (norms_ready = false on the first sub-chunk only).
 dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                          const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                          const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out, void* ws,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool norms_ready = false) {
   if (d.n_q == 0) return DSA_OK;
   WsHeader* h = static_cast<WsHeader*>(ws);
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes);
@@ -95,8 +106,12 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
   // The selection goes to the caller's idx_out when given, else to the
   // workspace region after the score matrix.
   int32_t* idx = idx_out ? idx_out : layer_idx_region(ws, d);
-  cudaError_t e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
-  if (e == cudaSuccess) e = dsa::launch_key_norm_max(d, k_idx, h, st);
+  cudaError_t e = cudaSuccess;
+  if (!norms_ready) {
+    e = dsa::launch_key_norm_max(d, k_idx, h, st);
+    if (e == cudaSuccess) e = dsa::launch_attn_key_norm_max(d, latent, rope, h, st);
+  }
+  if (e == cudaSuccess) e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
@@ -187,8 +202,10 @@ dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const u
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = clear_header(ws, st)) != DSA_OK) return s;
   if (d->n_q == 0) return DSA_OK;
-  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, false,
-                                           static_cast<WsHeader*>(ws), st));
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  cudaError_t e = dsa::launch_attn_key_norm_max(*d, latent, rope, h, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, false, h, st));
 }
 
 dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
@@ -274,7 +291,7 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const ui
     s = enqueue_layer(sub, dev->q + o * q_row, dev->latent, dev->rope, dev->q_idx + o * qi_row,
                       dev->k_idx, dev->w_idx + o * w_row, dev->out + o * o_row,
                       lse ? dev->lse + o * l_row : nullptr, idx_out ? dev->idx + o * i_row : nullptr,
-                      ws, s_run);
+                      ws, s_run, /*norms_ready=*/r0 > 0);
     if (s != DSA_OK) return s;
     e = cudaEventRecord(ev_b, s_run);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_b, 0);
@@ -323,7 +340,7 @@ const char* dsa_status_string(dsa_status s) {
     case DSA_ERR_TIMEOUT: return "a device-side bounded wait gave up";
     case DSA_ERR_CUDA: return "CUDA runtime or launch error";
     case DSA_ERR_DEVICE: return "current device is not an sm_100 (B200) GPU";
-    case DSA_ERR_RANGE: return "a selected index was outside the causal range";
+    case DSA_ERR_RANGE: return "a selected index was outside the causal range 0..t of its query";
     case DSA_ERR_SCRATCH_LIMIT:
       return "the chunk needs more scratch than the no-alloc entry point's static array holds";
     default: return "unknown status";

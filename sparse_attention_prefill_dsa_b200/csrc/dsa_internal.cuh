@@ -32,6 +32,27 @@ __device__ __forceinline__ void report(WsHeader* ws, unsigned int code, unsigned
   if (atomicCAS(&ws->status, 0u, code) == 0u) ws->status_info = info;
 }
 
+// Bounds checks of the checking build (compiled with -DDSA_CHECK=1, shipped
+// as libdsa_check.so): an index outside its buffer records kDevInternal with
+// kCheckSiteBase + site as the failing site, and the caller skips the access.
+// This stands in for a memory checker: nothing traps, and the status is read
+// like any other device-side failure. In the normal build every check is the
+// constant true and compiles away.
+constexpr unsigned int kCheckSiteBase = 1000;
+__device__ __forceinline__ bool check_bound(WsHeader* ws, long long i, long long cap,
+                                            unsigned int site) {
+  if (i >= 0 && i < cap) return true;
+  report(ws, kDevInternal, kCheckSiteBase + site);
+  return false;
+}
+#if defined(DSA_CHECK) && DSA_CHECK
+#define DSA_IN_BOUNDS(ws, i, cap, site) \
+  ::dsa::check_bound((ws), static_cast<long long>(i), static_cast<long long>(cap), (site))
+#else
+#define DSA_IN_BOUNDS(ws, i, cap, site) true
+#endif
+
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
   return __uint_as_float(static_cast<unsigned int>(h) << 16);
 }
@@ -57,11 +78,19 @@ cudaError_t launch_key_norm_max(const dsa_dims& d, const uint16_t* k_idx, WsHead
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld,
                         const uint16_t* q_idx, const uint16_t* k_idx, const float* w_idx,
                         int32_t* idx, WsHeader* ws, cudaStream_t st);
+// max_s ||[latent_s, rope_s]|| into the header, read by launch_sparse_attn's
+// kernel (launch it first, on the same stream, with the header's field zero).
+cudaError_t launch_attn_key_norm_max(const dsa_dims& d, const uint16_t* latent, const uint16_t* rope,
+                                     WsHeader* ws, cudaStream_t st);
 // prefix_valid: every idx row holds its min(top_k, t+1) valid keys first (as the
 // selections of dsa_topk_select do), so tiles past them are skipped.
 cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,
                                float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st);
+
+// DSA_OK when the current device is an sm_100 GPU, else DSA_ERR_DEVICE (or
+// DSA_ERR_CUDA when the runtime cannot say). Cached per device.
+dsa_status check_current_device();
 
 // The bounded-wait self-test (one CTA, two warps on mbarriers nothing signals).
 cudaError_t launch_bounded_wait_selftest(WsHeader* ws, long long* cycles, cudaStream_t st);

@@ -14,20 +14,25 @@
 // Rules of the static scratch:
 //  * it holds kNoallocScratchBytes (32 MiB) on every GPU that loads the
 //    library, until the process exits;
-//  * its device address is looked up once per device, on the first call made
-//    with that device current (that call should come before any stream
-//    capture);
+//  * its device address is looked up on the first call made with a device
+//    current, and again on the first call after that device's context was
+//    destroyed and created anew (cudaDeviceReset, or the primary context
+//    released and retained again), since the module and the array may then
+//    sit elsewhere; those calls should come before any stream capture;
 //  * every call on a device uses the same array, so calls that overlap on the
 //    GPU (different streams, or different host threads without ordering) race
 //    on it; the layer clears its status word and scalars itself at the start
 //    of each call, and every score it reads was written earlier in the same
 //    call.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include <mutex>
 
 #include "dsa.h"
+#include "dsa_internal.cuh"
 
 namespace {
 
@@ -38,6 +43,33 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];  // id of the context the address belongs to
+
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_once;
+
+void resolve_driver() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+}
+
+// Unique id of the current context (0 when it cannot be read).
+unsigned long long current_context_id() {
+  std::call_once(g_once, resolve_driver);
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!g_ctx_current || !g_ctx_id || g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      g_ctx_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_noalloc_scratch on the current device (host code only
 // sees a host-side stand-in for the symbol, never its device address).
@@ -45,14 +77,16 @@ dsa_status scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_DEVICE;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();  // reset the runtime's last-error state after the failed lookup
       return DSA_ERR_CUDA;
     }
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return DSA_OK;
@@ -75,6 +109,8 @@ extern "C" dsa_status dsa_prefill_layer_noalloc(const dsa_dims* dims, const uint
   if (dsa_workspace_size(dims, DSA_WS_LAYER) > kNoallocScratchBytes) return DSA_ERR_SCRATCH_LIMIT;
   if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u) != 0)
     return DSA_ERR_ALIGN;
+  // a GPU this library was not built for fails here, before the symbol lookup
+  if ((s = dsa::check_current_device()) != DSA_OK) return s;
   void* scratch = nullptr;
   s = scratch_for_current_device(&scratch);
   if (s != DSA_OK) return s;

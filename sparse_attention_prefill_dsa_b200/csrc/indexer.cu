@@ -13,18 +13,25 @@
 // writes 32 consecutive keys of a query row (128 coalesced bytes).
 //
 // Persistent, warp-specialised CTA (one per SM, 320 threads):
-//   warp 0      TMA producer: the block's q_idx rows (once per work unit) and
-//               a 4-stage ring of key tiles, 128-byte (or 64-byte) swizzled,
-//               plus the block's head weights into a double-buffered slot;
-//   warp 1      TMEM owner and single-thread MMA issuer (tcgen05.mma kind::f16,
-//               bf16 x bf16 -> f32), accumulating each tile into one of two
-//               256-column TMEM buffers;
+//   warp 0      TMA producer: takes work units from a queue (an atomic
+//               counter in the workspace header, reset before each launch),
+//               hands each unit to the other warps through a four-slot ring
+//               in shared memory (a -1 ends the stream), and loads the
+//               block's q_idx rows (once per unit), a 4-stage ring of key
+//               tiles, 128-byte (or 64-byte) swizzled, and the block's head
+//               weights into a double-buffered slot;
+//   warp 1      TMEM owner and MMA issuer (tcgen05.mma kind::f16, bf16 x bf16
+//               -> f32), issued warp-collectively by one elected lane with
+//               base descriptors plus compile-time offsets, accumulating each
+//               tile into one of two 256-column TMEM buffers;
 //   warps 2-9   epilogue: two warpgroups split the 256 columns; each thread
 //               reads its key's columns with tcgen05.ld and writes the scores.
-// A work unit is (query block, up to 32 consecutive causal key tiles); CTAs
-// take units round-robin. Key tiles past the last query of a block are never
-// loaded (causal skip); rows of a partial tile past the context read as zero
-// and no score past t is written.
+// A work unit is (query block, up to 32 consecutive causal key tiles). The
+// queue hands units out in slot-major order with the later (longer) query
+// blocks first, so every block's first 32 tiles go out before any block's
+// second and the units come roughly longest first. Key tiles past the last
+// query of a block are never loaded (causal skip); rows of a partial tile
+// past the context read as zero and no score past t is written.
 // Every wait is bounded: on a timeout the CTA records DSA_ERR_TIMEOUT in the
 // workspace, all roles stop, outstanding TMA loads and MMAs are drained, and
 // TMEM is freed before the CTA exits.
@@ -350,7 +357,8 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
               for (int j = 0; j < HI; ++j)
                 acc = fmaf(wv[qq * HI + j], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f), acc);
               const int i = qb * C::kQB + (col0 + qq * HI) / HI;
-              if (i < p.n_q && s <= p.q_pos0 + i) p.scores[static_cast<int64_t>(i) * p.ld + s] = acc;
+              if (i < p.n_q && s <= p.q_pos0 + i && DSA_IN_BOUNDS(p.ws, s, p.ld, 20))
+                p.scores[static_cast<int64_t>(i) * p.ld + s] = acc;
             }
           }
         }

@@ -241,7 +241,7 @@ struct Bucketer {
 // strictly larger. Uses hist[kBins] and cand[kCandCap]. Returns false if the
 // search did not settle (not expected; reported by the caller).
 __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vmax, int* hist,
-                            float* cand, Scratch& sm, float* vk_out, int* n_above) {
+                            float* cand, Scratch& sm, float* vk_out, int* n_above, WsHeader* ws) {
   float L = vmin, U = vmax;
   int kr = k, above = 0;
   int beg, end;
@@ -257,7 +257,10 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
     __syncthreads();
     const Bucketer bucket(L, U);
     for_segment(sc, beg, end, [&](int, float v) {
-      if (v >= L && v <= U) atomicAdd(&hist[bucket(v)], 1);
+      if (v >= L && v <= U) {
+        const int b = bucket(v);
+        if (DSA_IN_BOUNDS(ws, b, kBins, 1)) atomicAdd(&hist[b], 1);
+      }
     });
     __syncthreads();
     int ab;
@@ -269,7 +272,10 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
     if (c <= kCandCap) {
       // the bucket's members into cand[] (complete after the barrier)
       for_segment(sc, beg, end, [&](int, float v) {
-        if (v >= L && v <= U && bucket(v) == bstar) cand[atomicAdd(&sm.bc[2], 1)] = v;
+        if (v >= L && v <= U && bucket(v) == bstar) {
+          const int pos = atomicAdd(&sm.bc[2], 1);
+          if (DSA_IN_BOUNDS(ws, pos, kCandCap, 2)) cand[pos] = v;
+        }
       });
       __syncthreads();
     } else {
@@ -341,7 +347,7 @@ __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int
     bool keep = c == kAbove;
     if (c == kTie) keep = ties_before++ < need_ties;
     if (keep) {
-      if (pos < k) stage[pos] = s;  // never write past the row
+      if (pos < k) stage[pos] = s;  // never write past the row (a count mismatch is reported below)
       ++pos;
     }
   });
@@ -519,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         const int pr = l0 + 32 * t;
-        if (j < a.HI && pr < wpr) {
+        if (j < a.HI && pr < wpr && DSA_IN_BOUNDS(a.ws, j * qstride + 2 * pr + 1, kQRowBytes / 4, 3)) {
           const uint32_t v = qv[u][t];
           const double lo = static_cast<double>(__uint_as_float(v << 16));
           const double hi = static_cast<double>(__uint_as_float(v & 0xFFFF0000u));
@@ -561,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
   float vk;
   int n_above;
-  if (!kth_largest(sc, n, k, mn, mx, hist, cand, sm, &vk, &n_above)) {
+  if (!kth_largest(sc, n, k, mn, mx, hist, cand, sm, &vk, &n_above, a.ws)) {
     if (threadIdx.x == 0) report(a.ws, kDevInternal, static_cast<unsigned>(row));
     return;
   }
@@ -655,7 +661,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
                                 : make_uint2(0u, 0u);
       const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
                                   : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
-      if (lane < 4 && b + lane < tot_band) bx[b + lane] = d2key(xl);
+      if (lane < 4 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, a.bcap, 4))
+        bx[b + lane] = d2key(xl);
 #pragma unroll
       for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
     }
@@ -682,7 +689,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       for (int e = 0; e < 4; ++e) rank[e] = __reduce_add_sync(0xffffffffu, rank[e]);
       const int my_rank = lane == 0 ? rank[0] : lane == 1 ? rank[1] : lane == 2 ? rank[2] : rank[3];
       const int my_s = lane == 0 ? sb[0] : lane == 1 ? sb[1] : lane == 2 ? sb[2] : sb[3];
-      if (lane < 4 && b0 + lane < tot_band) sc[my_s] = my_rank < r ? INFINITY : -INFINITY;
+      if (lane < 4 && b0 + lane < tot_band && DSA_IN_BOUNDS(a.ws, my_s, n, 5))
+        sc[my_s] = my_rank < r ? INFINITY : -INFINITY;
     }
     const bool counted = __syncthreads_or(c_band > 2) == 0;
     const int kept = c_in + (bk0 >= 0 && sc[bk0] > hi_f) + (bk1 >= 0 && sc[bk1] > hi_f);
@@ -705,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     unsigned long long nb64;
     const int j = static_cast<int>(block_excl_scan64(static_cast<unsigned long long>(flag), &nb64, sm));
     const int nb = static_cast<int>(nb64);
-    if (flag) tile_s[j] = s;
+    if (flag && DSA_IN_BOUNDS(a.ws, j, kThreads, 6)) tile_s[j] = s;
     __syncthreads();
     for (int jj = warp < kw ? 4 * warp : nb; jj < nb; jj += 4 * kw) {
       uint2 raw[4];
@@ -727,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       const int nb = band_window(base);
       if (static_cast<int>(threadIdx.x) < nb) {
         const unsigned long long key = d2key(tile_x[threadIdx.x]);
-        if ((key & msk) == pre) atomicAdd(&hist256[static_cast<int>((key >> shift) & 0xFFull)], 1);
+        const int hb = static_cast<int>((key >> shift) & 0xFFull);
+        if ((key & msk) == pre && DSA_IN_BOUNDS(a.ws, hb, 256, 7)) atomicAdd(&hist256[hb], 1);
       }
       __syncthreads();
     }
@@ -843,13 +852,16 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   } else if (static_cast<size_t>(max_smem) < bytes + static_bytes) {
     return cudaErrorInvalidConfiguration;
   }
+  cudaError_t e;
   if (refine) {
-    cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(bytes));
+    e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes));
+    if (e != cudaSuccess) return e;
     topk_kernel<true><<<d.n_q, kThreads, bytes, st>>>(a);
   } else {
-    cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(bytes));
+    e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes));
+    if (e != cudaSuccess) return e;
     topk_kernel<false><<<d.n_q, kThreads, bytes, st>>>(a);
   }
   return cudaGetLastError();

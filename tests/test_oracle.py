@@ -328,3 +328,41 @@ def test_tie_stress_workload_selection_is_lexsort(oracle_lib):
         kth = np.sort(sc[i, : t + 1])[::-1][d.top_k - 1]
         n_tied += int((sc[i, : t + 1] == kth).sum())
     assert n_tied > 4 * d.n_q  # the recipe really produces ties at the boundary
+
+
+# ------------------------------------------------ stored selection digests
+
+
+def test_stored_selection_digests_match_the_oracle():
+    """tests/golden/selection_hashes.json was written by an oracle-only
+    script; recompute the tiny workload whole and a few 256-row blocks of the
+    others here, so the stored digests stay tied to the oracle as it is."""
+    import importlib.util
+
+    here = os.path.join(os.path.dirname(__file__), "golden")
+    spec = importlib.util.spec_from_file_location(
+        "make_selection_hashes", os.path.join(here, "make_selection_hashes.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with open(os.path.join(here, "selection_hashes.json")) as f:
+        g = json.load(f)
+    nb = g["block_rows"]
+    assert set(g["cases"]) == {mod.case_key(*c) for c in mod.CASES}
+    for key, c in sorted(g["cases"].items()):
+        d, x = workloads.workload_inputs(c["workload"], c["w_mode"])
+        assert mod.inputs_digest(x) == c["inputs_sha256"], key
+        n_blocks = (d.n_q + nb - 1) // nb
+        assert len(c["block_sha256"]) == n_blocks
+        if d.n_q <= nb:
+            whole, _ = mod.selection_digests(mod.oracle_selection(d, x))
+            assert whole == c["selection_sha256"], key
+            continue
+        # first block always; the last one too where the oracle is quick
+        blocks = [0] if d.ctx_len > 20000 else [0, n_blocks - 1]
+        for b in blocks:
+            rows = np.arange(b * nb, min(d.n_q, (b + 1) * nb), dtype=np.int32)
+            if d.ctx_len > 20000:
+                rows = rows[:nb]
+            sel = mod.oracle_selection(d, x, rows=rows)
+            _, digests = mod.selection_digests(sel)
+            assert digests[0] == c["block_sha256"][b], (key, b)

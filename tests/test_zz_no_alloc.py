@@ -10,7 +10,7 @@ import pytest
 import workloads
 from workloads import make_dims
 
-from dsa_test_util import assert_attn_close, empty_bf16, host_bf16_as_f32, run_layer, stage
+from dsa_test_util import empty_bf16, host_bf16_as_f32, run_layer, stage
 
 pytestmark = pytest.mark.gpu
 
@@ -50,14 +50,42 @@ def _reduced_chunk():
 
 
 def test_noalloc_matches_layer_on_two_calls_in_a_row(dsa):
+    """Both calls run the same kernels on the same inputs, so the results are
+    the same bits, not merely within the attention tolerance."""
     cases = [workloads.workload_inputs("tiny_256q"), _reduced_chunk()]
     staged = [(d, stage(x)) for d, x in cases]
     results = [_noalloc(dsa, d, xd) for d, xd in staged]  # two calls in a row
     for (d, xd), (out, lse, idx) in zip(staged, results):
         ref_out, ref_lse, ref_idx = run_layer(dsa, d, xd)
         assert np.array_equal(idx, ref_idx)
-        assert_attn_close(out, ref_out.astype(np.float64))
-        np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=2e-3)
+        assert np.array_equal(out, ref_out)
+        assert np.array_equal(lse, ref_lse)
+
+
+def _scratch_bytes(n_q, T, k):
+    return 256 + n_q * ((T + 127) // 128 * 128 + k) * 4
+
+
+def test_noalloc_at_its_scratch_limit(dsa):
+    """1,024 queries at top_k 2048 fit up to a 6,016-token context: the
+    largest such chunk runs (bit-identical to dsa_prefill_layer); one more
+    token needs 128 more score columns per row and is refused."""
+    import torch
+
+    fits = make_dims(1024, 6016 - 1024, 6016, 32, 512, 64, 32, 128, 2048)
+    over = make_dims(1024, 6017 - 1024, 6017, 32, 512, 64, 32, 128, 2048)
+    assert _scratch_bytes(1024, 6016, 2048) <= dsa.DSA_NOALLOC_SCRATCH_BYTES
+    assert _scratch_bytes(1024, 6017, 2048) > dsa.DSA_NOALLOC_SCRATCH_BYTES
+    assert dsa.dsa_workspace_size(fits, dsa.DSA_WS_LAYER) == _scratch_bytes(1024, 6016, 2048)
+    xd = stage(workloads.generate(fits, 78, "normal", "uniform"))
+    out, lse, idx = _noalloc(dsa, fits, xd)
+    ref_out, ref_lse, ref_idx = run_layer(dsa, fits, xd)
+    assert np.array_equal(idx, ref_idx) and np.array_equal(out, ref_out)
+    assert np.array_equal(lse, ref_lse)
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(16, dtype=torch.float32, device="cuda")
+    assert (dsa.dsa_prefill_layer_noalloc(over, x, x, x, x, x, w, x, None, None, None)
+            == dsa.DSA_ERR_SCRATCH_LIMIT)
 
 
 def test_noalloc_refuses_chunks_beyond_its_scratch(dsa):
