@@ -85,6 +85,8 @@ typedef int32_t dsa_status;
 #define DSA_WS_TOPK 1
 #define DSA_WS_ATTN 2
 #define DSA_WS_LAYER 3
+#define DSA_WS_DECODE_ATTN 4
+#define DSA_WS_DECODE_LAYER 5
 
 /* Bytes of device workspace the call `which` needs for these dims (0 on bad
  * arguments). The first 256 bytes of every workspace hold the device status
@@ -163,6 +165,35 @@ dsa_status dsa_prefill_layer(const dsa_dims* dims, const uint16_t* q, const uint
                              const uint16_t* k_idx, const float* w_idx, uint16_t* out,
                              float* lse, int32_t* idx_out, void* workspace,
                              size_t workspace_bytes, void* stream);
+
+/* Decode-side attention: dsa_sparse_attn_prefill for chunks of few queries (a
+ * decode step is n_q = 1). The per-query kernel runs one query per SM, so a
+ * chunk smaller than the GPU would leave most SMs idle; here each query's
+ * selected keys are cut into up to ceil(top_k / 128) ranges of 128-key tiles
+ * (n_split = min(ceil(top_k / 128), SMs / n_q), at least 1) that run on
+ * different SMs, each writing its unnormalised partial output, reference
+ * maximum and row sum to the workspace; a combine pass then merges them
+ * (flash-decoding style: out = sum_j 2^(m_j - M) O_j / sum_j 2^(m_j - M) l_j).
+ * Same definition, arguments, layouts and errors as dsa_sparse_attn_prefill,
+ * with a workspace of dsa_workspace_size(dims, DSA_WS_DECODE_ATTN) bytes.
+ * Results agree with dsa_sparse_attn_prefill within rounding (the sums are
+ * grouped differently), and depend on n_q through n_split. The feedman.me
+ * post profiles prefill only; this call is the decode side of the same
+ * layer (its component table lists decode throughput for the same model). */
+dsa_status dsa_sparse_attn_decode(const dsa_dims* dims, const uint16_t* q,
+                                  const uint16_t* latent, const uint16_t* rope,
+                                  const int32_t* idx, uint16_t* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* The whole layer for a decode step (few queries): dsa_prefill_layer with the
+ * attention of dsa_sparse_attn_decode. The indexer spreads a small chunk's key
+ * tiles over all SMs in either call. Workspace: dsa_workspace_size(dims,
+ * DSA_WS_DECODE_LAYER) bytes. Selections are those of dsa_prefill_layer (bit
+ * for bit); outputs agree with it within rounding. */
+dsa_status dsa_decode_layer(const dsa_dims* dims, const uint16_t* q, const uint16_t* latent,
+                            const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
+                            const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* Device copies of the layer's tensors for dsa_prefill_layer_host, owned by
  * the caller, each of the full size given under dsa_prefill_layer and 16-byte

@@ -42,6 +42,8 @@ DSA_WS_INDEX_SCORES = 0
 DSA_WS_TOPK = 1
 DSA_WS_ATTN = 2
 DSA_WS_LAYER = 3
+DSA_WS_DECODE_ATTN = 4
+DSA_WS_DECODE_LAYER = 5
 
 DSA_MAX_TOPK = 2048
 DSA_MAX_CTX = 49152
@@ -49,7 +51,8 @@ DSA_MAX_CTX = 49152
 EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",
             "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host",
-            "dsa_selftest_bounded_wait", "dsa_partition_queries")
+            "dsa_selftest_bounded_wait", "dsa_partition_queries", "dsa_sparse_attn_decode",
+            "dsa_decode_layer")
 
 
 class dsa_dims(ctypes.Structure):
@@ -101,6 +104,9 @@ def library():
     lib.dsa_sparse_attn_prefill.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     lib.dsa_prefill_layer.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]
+    lib.dsa_sparse_attn_decode.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.dsa_decode_layer.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                     ctypes.c_size_t, _P]
     lib.dsa_prefill_layer_noalloc.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.dsa_prefill_layer_host.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
@@ -112,7 +118,8 @@ def library():
     lib.dsa_status_string.restype = ctypes.c_char_p
     for f in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
               "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc",
-              "dsa_prefill_layer_host", "dsa_selftest_bounded_wait", "dsa_partition_queries"):
+              "dsa_prefill_layer_host", "dsa_selftest_bounded_wait", "dsa_partition_queries",
+              "dsa_sparse_attn_decode", "dsa_decode_layer"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -185,6 +192,21 @@ def dsa_prefill_layer(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_
                                   _p(k_idx), _p(w_idx), _p(out), _p(lse), _p(idx_out),
                                   _p(workspace), _nbytes(workspace, workspace_bytes),
                                   _stream(stream))
+
+
+def dsa_sparse_attn_decode(dims, q, latent, rope, idx, out, lse, workspace, workspace_bytes=None,
+                           stream=None) -> int:
+    return library().dsa_sparse_attn_decode(_dims(dims), _p(q), _p(latent), _p(rope), _p(idx),
+                                            _p(out), _p(lse), _p(workspace),
+                                            _nbytes(workspace, workspace_bytes), _stream(stream))
+
+
+def dsa_decode_layer(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out, workspace,
+                     workspace_bytes=None, stream=None) -> int:
+    return library().dsa_decode_layer(_dims(dims), _p(q), _p(latent), _p(rope), _p(q_idx),
+                                      _p(k_idx), _p(w_idx), _p(out), _p(lse), _p(idx_out),
+                                      _p(workspace), _nbytes(workspace, workspace_bytes),
+                                      _stream(stream))
 
 
 def dsa_prefill_layer_noalloc(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out,

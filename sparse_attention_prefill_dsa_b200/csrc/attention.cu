@@ -133,6 +133,15 @@ struct AttnParams {
   int prefix_valid;  // idx rows hold min(k, t+1) valid keys first (selections of this library)
   float scale_log2;  // softmax_scale * log2(e)
   WsHeader* ws;
+  // Work items: item w is query w / n_split and the key tiles [j * tps,
+  // (j + 1) * tps) of its selection, j = w % n_split. n_split = 1 (one item
+  // per query) writes out / lse directly; n_split > 1 (decode: few queries,
+  // their tiles spread over SMs) writes each item's unnormalised partial O,
+  // running maximum (log2 units) and row sum to part_o / part_ml for the
+  // combine pass.
+  int n_split, tps, n_items;
+  float* part_o;   // [n_items, H, DC]
+  float2* part_ml; // [n_items, H]: (m, l)
 };
 
 __device__ __forceinline__ int n_valid_of(const AttnParams& p, int i) {
@@ -146,6 +155,42 @@ __device__ __forceinline__ int n_tiles_of(const AttnParams& p, int i) {
 // Selected key `sel` of query i, or -1 past the query's selection.
 __device__ __forceinline__ int selected_row(const AttnParams& p, int i, int sel) {
   return sel < n_valid_of(p, i) ? __ldg(p.idx + static_cast<int64_t>(i) * p.k + sel) : -1;
+}
+
+// Query and key-tile range [t0, t1) of item w.
+__device__ __forceinline__ void item_range(const AttnParams& p, int w, int& i, int& t0, int& t1) {
+  i = w / p.n_split;
+  t0 = (w - i * p.n_split) * p.tps;
+  t1 = min(n_tiles_of(p, i), t0 + p.tps);
+}
+
+// This CTA's first item at or after w (w, w + grid, ...) with at least one
+// key tile, or n_items. Every role walks the same sequence.
+__device__ __forceinline__ int next_item(const AttnParams& p, int w) {
+  for (; w < p.n_items; w += gridDim.x) {
+    int i, t0, t1;
+    item_range(p, w, i, t0, t1);
+    if (t0 < t1) return w;
+  }
+  return p.n_items;
+}
+
+// The tile after tile j of item w (query i, tiles up to t1): (i, j + 1), or
+// the first tile of this CTA's next item; ni = -1 when there is none.
+__device__ __forceinline__ void tile_after(const AttnParams& p, int w, int i, int j, int t1, int& ni,
+                                           int& nj) {
+  if (j + 1 < t1) {
+    ni = i;
+    nj = j + 1;
+    return;
+  }
+  const int nw = next_item(p, w + static_cast<int>(gridDim.x));
+  ni = -1;
+  nj = 0;
+  if (nw < p.n_items) {
+    int e1;
+    item_range(p, nw, ni, nj, e1);
+  }
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -374,18 +419,22 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       doff[e] = key * 128 + ((part ^ (key & 7)) << 4);
     }
     int cur[R], nxt[R];
-    if (blockIdx.x < p.n_q) {
+    const int w0 = next_item(p, blockIdx.x);
+    if (w0 < p.n_items) {
+      int i0, a0, b0;
+      item_range(p, w0, i0, a0, b0);
 #pragma unroll
-      for (int e = 0; e < R; ++e) cur[e] = selected_row(p, blockIdx.x, kbase + 4 * e);
+      for (int e = 0; e < R; ++e) cur[e] = selected_row(p, i0, a0 * 128 + kbase + 4 * e);
     }
     uint32_t tc = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x) {
-      const int nt = n_tiles_of(p, i);
-      for (int j = 0; j < nt && ok; ++j, ++tc) {
-        const int ni = j + 1 < nt ? i : i + gridDim.x;
-        const int nj = j + 1 < nt ? j + 1 : 0;
-        if (ni < p.n_q) {
+    for (int w = w0; w < p.n_items && ok; w = next_item(p, w + gridDim.x)) {
+      int i, t0, t1;
+      item_range(p, w, i, t0, t1);
+      for (int j = t0; j < t1 && ok; ++j, ++tc) {
+        int ni, nj;
+        tile_after(p, w, i, j, t1, ni, nj);
+        if (ni >= 0) {
 #pragma unroll
           for (int e = 0; e < R; ++e) nxt[e] = selected_row(p, ni, nj * 128 + kbase + 4 * e);
         }
@@ -450,12 +499,13 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     uint32_t pend_tc = 0, pend_qi = 0;
     uint32_t tc = 0, qi = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
-      const int nt = n_tiles_of(p, i);
-      for (int j = 0; j < nt; ++j, ++tc) {
+    for (int w = next_item(p, blockIdx.x); w < p.n_items && ok; w = next_item(p, w + gridDim.x), ++qi) {
+      int i, t0, t1;
+      item_range(p, w, i, t0, t1);
+      for (int j = t0; j < t1; ++j, ++tc) {
         const int sb = tc & 1;
         const uint32_t d_s = tmem_base + C::kTmemS + sb * NH;
-        if (j == 0) {
+        if (j == t0) {
           // a new query: the previous query's last PV goes first, then q
           if (pend && !(ok = attn_pv<C>(p, abort_flag, bars, tmem_base, dpair_mn, dp, pend_tc, pend_qi,
                                         pend_first, pend_last)))
@@ -485,8 +535,8 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         pend = true;
         pend_tc = tc;
         pend_qi = qi;
-        pend_first = j == 0;
-        pend_last = j == nt - 1;
+        pend_first = j == t0;
+        pend_last = j == t1 - 1;
       }
     }
     if (ok && pend)
@@ -503,26 +553,34 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const bool q_loader = warp == 5 && lane == 0;
     int q_loads = 0;
-    if (q_loader && blockIdx.x < p.n_q) {
-      prefetch_tmap(&tm_q);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-      for (int c = 0; c < C::kQChunks; ++c)
-        tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, blockIdx.x * H, q_full);
-      q_loads = 1;
+    const int w_first = next_item(p, blockIdx.x);
+    int row_next = -1;
+    if (w_first < p.n_items) {
+      int i0, a0, b0;
+      item_range(p, w_first, i0, a0, b0);
+      row_next = selected_row(p, i0, a0 * 128 + r);
+      if (q_loader) {
+        prefetch_tmap(&tm_q);
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
+        for (int c = 0; c < C::kQChunks; ++c)
+          tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, i0 * H, q_full);
+        q_loads = 1;
+      }
     }
     uint32_t tc = 0, qi = 0, xc = 0;
     bool ok = true;
-    int row_next = blockIdx.x < p.n_q ? selected_row(p, blockIdx.x, r) : -1;
     // max_s ||k_s|| of the context, with the rounding slack of its float32 sum
     const float kmax = __uint_as_float(*reinterpret_cast<volatile unsigned int*>(&p.ws->akmax_bits));
     const float bound_scale = fabsf(p.scale_log2) * kmax;
     // the exchange slot of head h (lane) from the warp of quarter-rank qq of
     // h's half: warps hh*4 .. hh*4+3 hold the halves' partial values
     const int xslot = (lane / HH) * 4 * 16 + (lane % HH);
-    for (int i = blockIdx.x; i < p.n_q && ok; i += gridDim.x, ++qi) {
-      const int nt = n_tiles_of(p, i);
+    for (int w = w_first; w < p.n_items && ok; w = next_item(p, w + gridDim.x), ++qi) {
+      int i, t0, t1;
+      item_range(p, w, i, t0, t1);
       const int ob = qi & 1;
-      const bool next_q = i + static_cast<int>(gridDim.x) < p.n_q;
+      const int w_next = next_item(p, w + gridDim.x);
+      const bool next_q = w_next < p.n_items;
       float m_lane = -INFINITY;       // running max (log2 units) of head `lane` (all heads)
       float bound_lane = INFINITY;    // B_lane: bound on every score of head `lane`
       bool fixed_m = false;           // B_h <= m_h + 64 for every head: keep m as it is
@@ -532,13 +590,13 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       __syncwarp();
 #pragma unroll
       for (int h = 0; h < HH; ++h) lpart[h] = 0.f;
-      for (int j = 0; j < nt; ++j, ++tc) {
+      for (int j = t0; j < t1; ++j, ++tc) {
         const int sb = tc & 1;
         const int row = row_next;
         {
-          const int ni = j + 1 < nt ? i : i + static_cast<int>(gridDim.x);
-          const int nj = j + 1 < nt ? j + 1 : 0;
-          row_next = ni < p.n_q ? selected_row(p, ni, nj * 128 + r) : -1;
+          int ni, nj;
+          tile_after(p, w, i, j, t1, ni, nj);
+          row_next = ni >= 0 ? selected_row(p, ni, nj * 128 + r) : -1;
         }
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (tc >> 1) & 1, abort_flag, p.ws, 40));
         if (!ok) break;
@@ -547,7 +605,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
         tmem_ld_row<HH>(tmem_base + lane_addr + C::kTmemS + sb * NH + hh * HH, x);
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
-        if (j == 0) {
+        if (j == t0) {
           // this warp's share of ||q_h||^2 for every head (q chunks sw, sw+8;
           // lane = head), reading a row's 16-byte units in a lane-rotated order
           ok = __all_sync(0xffffffffu, mbar_wait(q_full, qi & 1, abort_flag, p.ws, 46));
@@ -570,7 +628,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           }
           sNorm[sw * 32 + lane] = qn2;
         }
-        const bool issue_q = j == nt - 1 && q_loader && next_q;
+        const bool issue_q = j == t1 - 1 && q_loader && next_q;
         const bool valid = row >= 0 && row <= p.q_pos0 + i;
         if (!fixed_m) {
           // per-head maximum of this tile over all 128 keys (log2 units)
@@ -588,7 +646,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           float tmax = -INFINITY;
           if (lane < NH)
             tmax = fmaxf(fmaxf(xbuf[xslot], xbuf[xslot + 16]), fmaxf(xbuf[xslot + 32], xbuf[xslot + 48]));
-          if (j == 0 && lane < NH) {
+          if (j == t0 && lane < NH) {
             float qn2 = 0.f;
 #pragma unroll
             for (int w = 0; w < C::kSoftmaxWarps; ++w) qn2 += sNorm[w * 32 + lane];
@@ -608,7 +666,7 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
             }
             mrep[lane] = m_lane;
             __syncwarp();
-            if (j > 0) {  // rescale this warp's O^T columns once the previous tile's PV is complete
+            if (j > t0) {  // rescale this warp's O^T columns once the previous tile's PV is complete
               ok = __all_sync(0xffffffffu, mbar_wait(o_step, (tc - 1) & 1, abort_flag, p.ws, 42));
               if (!ok) break;
               tc_fence_after();
@@ -631,8 +689,10 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
           // every QK^T of query i has completed and every warp has read its q
           // rows (the first tile's exchange): bring in the next query's q
           mbar_arrive_expect_tx(q_full, C::kQBytes);
+          int i_next, a1, b1;
+          item_range(p, w_next, i_next, a1, b1);
           for (int c = 0; c < C::kQChunks; ++c)
-            tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, (i + gridDim.x) * H, q_full);
+            tma_load_2d(sQ + c * C::kQChunkBytes, &tm_q, c * 64, i_next * H, q_full);
           ++q_loads;
         }
         // the previous tile's PV has finished reading P
@@ -687,6 +747,30 @@ __global__ void __launch_bounds__(AttnCfg<H, DC, DR>::kThreads, 1)
       if (!ok) break;
       float l_lane = 0.f;
       if (lane < NH) l_lane = xbuf[xslot] + xbuf[xslot + 16] + xbuf[xslot + 32] + xbuf[xslot + 48];
+      if (p.n_split > 1) {
+        // a partial of a split query: unnormalised O, the reference maximum
+        // (log2 units) and the row sum, merged by the combine pass
+        if (sw == 0 && lane < H)
+          p.part_ml[static_cast<int64_t>(w) * H + lane] = make_float2(m_lane, l_lane);
+#pragma unroll 1
+        for (int mb = 0; mb < C::MB; ++mb) {
+          float o[HH];
+          tmem_ld_row<HH>(tmem_base + lane_addr + C::kTmemO + (ob * C::MB + mb) * NH + hh * HH, o);
+          const int d = mb * 128 + r;
+          if (d < DC) {
+            float* orow = p.part_o + (static_cast<int64_t>(w) * H + hh * HH) * DC + d;
+#pragma unroll
+            for (int h = 0; h < HH; ++h)
+              if (hh * HH + h < H &&
+                  DSA_IN_BOUNDS(p.ws, (static_cast<int64_t>(w) * H + hh * HH + h) * DC + d,
+                                static_cast<int64_t>(p.n_items) * H * DC, 15))
+                orow[h * DC] = o[h];
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&o_empty[ob]);
+        continue;
+      }
       const float inv_lane = l_lane > 0.f ? 1.f / l_lane : 0.f;
       if (sw == 0 && lane < H && p.lse)
         p.lse[static_cast<int64_t>(i) * H + lane] =
@@ -763,10 +847,52 @@ int num_sms() {
 
 constexpr int kOneCtaPerSmSmem = 120 * 1024;
 
+// Merges the partials of a split query, one CTA per (query, head), a thread
+// per 4 dims: with M the largest reference maximum of the query's items and
+// a_j = 2^(m_j - M), out = sum_j a_j O_j / sum_j a_j l_j and
+// lse = (M + log2 sum_j a_j l_j) ln 2. Items without tiles were never
+// written and are skipped, as are items whose keys were all masked (l = 0).
+template <int H, int DC>
+__global__ void attn_split_combine(const AttnParams p) {
+  const int i = blockIdx.x / H, h = blockIdx.x % H;
+  const int nt = n_tiles_of(p, i);
+  float M = -INFINITY;
+  for (int j = 0; j < p.n_split && j * p.tps < nt; ++j) {
+    const float2 ml = p.part_ml[(static_cast<int64_t>(i) * p.n_split + j) * H + h];
+    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  }
+  float L = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int d0 = threadIdx.x * 4;
+  for (int j = 0; j < p.n_split && j * p.tps < nt; ++j) {
+    const int64_t w = static_cast<int64_t>(i) * p.n_split + j;
+    const float2 ml = p.part_ml[w * H + h];
+    if (!(ml.y > 0.f)) continue;
+    const float a = exp2f(ml.x - M);
+    L = fmaf(a, ml.y, L);
+    if (d0 < DC) {
+      const float4 o = *reinterpret_cast<const float4*>(p.part_o + (w * H + h) * DC + d0);
+      acc[0] = fmaf(a, o.x, acc[0]);
+      acc[1] = fmaf(a, o.y, acc[1]);
+      acc[2] = fmaf(a, o.z, acc[2]);
+      acc[3] = fmaf(a, o.w, acc[3]);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (d0 < DC) {
+    uint16_t* orow = p.out + (static_cast<int64_t>(i) * H + h) * DC + d0;
+    const uint32_t lo = f32_to_bf16_rne(acc[0] * inv) | (static_cast<uint32_t>(f32_to_bf16_rne(acc[1] * inv)) << 16);
+    const uint32_t hi = f32_to_bf16_rne(acc[2] * inv) | (static_cast<uint32_t>(f32_to_bf16_rne(acc[3] * inv)) << 16);
+    *reinterpret_cast<uint2*>(orow) = make_uint2(lo, hi);
+  }
+  if (threadIdx.x == 0 && p.lse)
+    p.lse[static_cast<int64_t>(i) * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
 template <int H, int DC, int DR>
 cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                    const uint16_t* rope, const int32_t* idx, uint16_t* out, float* lse,
-                   bool prefix_valid, WsHeader* ws, cudaStream_t st) {
+                   bool prefix_valid, WsHeader* ws, int n_split, void* part, cudaStream_t st) {
   using C = AttnCfg<H, DC, DR>;
   AttnParams p;
   p.q = q;
@@ -782,16 +908,30 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
   p.prefix_valid = prefix_valid ? 1 : 0;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.ws = ws;
+  const int max_tiles = (d.top_k + 127) / 128;
+  p.n_split = n_split < 1 ? 1 : (n_split > max_tiles ? max_tiles : n_split);
+  p.tps = (max_tiles + p.n_split - 1) / p.n_split;
+  p.n_items = d.n_q * p.n_split;
+  p.part_ml = static_cast<float2*>(part);
+  p.part_o = part ? reinterpret_cast<float*>(static_cast<char*>(part) +
+                                              attn_split_ml_bytes(d.n_q, p.n_split, H))
+                  : nullptr;
+  if (p.n_split > 1 && !part) return cudaErrorInvalidValue;
   CUtensorMap tm_q;
   if (!make_tmap_bf16_2d(&tm_q, q, DC + DR, static_cast<uint64_t>(d.n_q) * H, 64, H,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const int grid = d.n_q < num_sms() ? d.n_q : num_sms();
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc<H, DC, DR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   sparse_attn_tc<H, DC, DR><<<grid, C::kThreads, smem, st>>>(tm_q, p);
+  if (p.n_split > 1) {
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_split_combine<H, DC><<<d.n_q * H, (DC / 4 + 31) / 32 * 32, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -816,12 +956,21 @@ cudaError_t launch_attn_key_norm_max(const dsa_dims& d, const uint16_t* latent, 
 
 cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,
-                               float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st) {
+                               float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st,
+                               int n_split, void* part) {
   if (d.n_heads == 32 && d.d_latent == 512 && d.d_rope == 64)
-    return launch<32, 512, 64>(d, q, latent, rope, idx, out, lse, prefix_valid, ws, st);
+    return launch<32, 512, 64>(d, q, latent, rope, idx, out, lse, prefix_valid, ws, n_split, part, st);
   if (d.n_heads == 4 && d.d_latent == 64 && d.d_rope == 16)
-    return launch<4, 64, 16>(d, q, latent, rope, idx, out, lse, prefix_valid, ws, st);
+    return launch<4, 64, 16>(d, q, latent, rope, idx, out, lse, prefix_valid, ws, n_split, part, st);
   return cudaErrorInvalidValue;
+}
+
+int attn_decode_split(const dsa_dims& d) {
+  const int max_tiles = (d.top_k + 127) / 128;
+  if (d.n_q <= 0) return 1;
+  int n = num_sms() / d.n_q;
+  if (n > max_tiles) n = max_tiles;
+  return n < 1 ? 1 : n;
 }
 
 }  // namespace dsa

@@ -76,6 +76,18 @@ int32_t* layer_idx_region(void* ws, const dsa_dims& d) {
                                     layer_scores_bytes(d));
 }
 
+size_t layer_bytes(const dsa_dims& d) {
+  return dsa::kWsHeaderBytes + layer_scores_bytes(d) +
+         (static_cast<size_t>(d.n_q) * d.top_k * sizeof(int32_t) + 255) / 256 * 256;
+}
+
+// decode: the split attention's partials follow the header (attention alone)
+// or the layer's score and selection regions (whole layer)
+size_t decode_part_bytes(const dsa_dims& d) {
+  const int n_split = dsa::attn_decode_split(d);
+  return n_split > 1 ? dsa::attn_split_bytes(d.n_q, n_split, d.n_heads, d.d_latent) : 0;
+}
+
 dsa_status check_ws(const dsa_dims& d, int which, void* ws, size_t bytes) {
   if (!ws) return DSA_ERR_WORKSPACE;
   if (!aligned16(ws)) return DSA_ERR_ALIGN;
@@ -98,7 +110,7 @@ dsa_status clear_header(void* ws, cudaStream_t st) {
 dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                          const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                          const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out, void* ws,
-                         cudaStream_t st, bool norms_ready = false) {
+                         cudaStream_t st, bool norms_ready = false, bool decode = false) {
   if (d.n_q == 0) return DSA_OK;
   WsHeader* h = static_cast<WsHeader*>(ws);
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes);
@@ -115,6 +127,12 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
+  if (decode) {
+    const int n_split = dsa::attn_decode_split(d);
+    void* part = n_split > 1 ? static_cast<char*>(ws) + layer_bytes(d) : nullptr;
+    return from_cuda(
+        dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, true, h, st, n_split, part));
+  }
   return from_cuda(dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, true, h, st));
 }
 
@@ -140,6 +158,10 @@ size_t dsa_workspace_size(const dsa_dims* d, int32_t which) {
     case DSA_WS_LAYER:
       return dsa::kWsHeaderBytes + layer_scores_bytes(*d) +
              static_cast<size_t>(d->n_q) * d->top_k * sizeof(int32_t);
+    case DSA_WS_DECODE_ATTN:
+      return dsa::kWsHeaderBytes + decode_part_bytes(*d);
+    case DSA_WS_DECODE_LAYER:
+      return layer_bytes(*d) + decode_part_bytes(*d);
     default:
       return 0;
   }
@@ -206,6 +228,48 @@ dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const u
   cudaError_t e = dsa::launch_attn_key_norm_max(*d, latent, rope, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, false, h, st));
+}
+
+dsa_status dsa_sparse_attn_decode(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
+                                  const uint16_t* rope, const int32_t* idx, uint16_t* out,
+                                  float* lse, void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_dims(d, true, false);
+  if (s != DSA_OK) return s;
+  if (!q || !latent || !rope || !idx || !out) return DSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(idx) ||
+      !aligned16(out) || (lse && !aligned16(lse)))
+    return DSA_ERR_ALIGN;
+  if ((s = check_ws(*d, DSA_WS_DECODE_ATTN, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  WsHeader* h = static_cast<WsHeader*>(ws);
+  cudaError_t e = dsa::launch_attn_key_norm_max(*d, latent, rope, h, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  const int n_split = dsa::attn_decode_split(*d);
+  void* part = n_split > 1 ? static_cast<char*>(ws) + dsa::kWsHeaderBytes : nullptr;
+  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, false, h, st,
+                                           n_split, part));
+}
+
+dsa_status dsa_decode_layer(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
+                            const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
+                            const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_dims(d, true, true);
+  if (s != DSA_OK) return s;
+  if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
+      !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(out) || (lse && !aligned16(lse)) ||
+      (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGN;
+  if ((s = check_ws(*d, DSA_WS_DECODE_LAYER, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  return enqueue_layer(*d, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out, ws, st,
+                       /*norms_ready=*/false, /*decode=*/true);
 }
 
 dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,

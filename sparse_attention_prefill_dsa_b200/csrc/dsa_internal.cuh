@@ -84,9 +84,23 @@ cudaError_t launch_attn_key_norm_max(const dsa_dims& d, const uint16_t* latent, 
                                      WsHeader* ws, cudaStream_t st);
 // prefix_valid: every idx row holds its min(top_k, t+1) valid keys first (as the
 // selections of dsa_topk_select do), so tiles past them are skipped.
+// n_split > 1 cuts every query's key tiles into n_split ranges on different
+// SMs (decode); `part` is then the partials' scratch of
+// attn_split_bytes(n_q, n_split, n_heads, d_latent) bytes, 16-byte aligned,
+// and a combine pass writes out / lse.
 cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,
-                               float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st);
+                               float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st,
+                               int n_split = 1, void* part = nullptr);
+// The split the decode entry points use: as many ranges per query as leave no
+// SM idle, at most one per 128-key tile of top_k.
+int attn_decode_split(const dsa_dims& d);
+inline size_t attn_split_ml_bytes(int n_q, int n_split, int H) {
+  return (static_cast<size_t>(n_q) * n_split * H * 8 + 255) / 256 * 256;
+}
+inline size_t attn_split_bytes(int n_q, int n_split, int H, int DC) {
+  return attn_split_ml_bytes(n_q, n_split, H) + static_cast<size_t>(n_q) * n_split * H * DC * 4;
+}
 
 // DSA_OK when the current device is an sm_100 GPU, else DSA_ERR_DEVICE (or
 // DSA_ERR_CUDA when the runtime cannot say). Cached per device.

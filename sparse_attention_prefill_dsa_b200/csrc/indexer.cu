@@ -66,7 +66,7 @@ struct IdxCfg {
   static constexpr int kStages = 4;
   static constexpr int kKSteps = DI / 16;
   static constexpr int kStepsPerChunk = kChunk / 16;
-  static constexpr int kTilesPerUnit = 32;
+  static constexpr int kTilesPerUnit = 32;             // key tiles per work unit (fewer for small chunks)
   static constexpr int kEpiWarps = 8;                  // warps 2-9
   static constexpr int kThreads = 32 * (2 + kEpiWarps);
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kM, kN, false, false);
@@ -88,7 +88,8 @@ struct IdxParams {
   float* scores;
   int64_t ld;
   int n_q, q_pos0;
-  int n_units, n_qb;  // units: n_qb query blocks x (up to) kTilesPerUnit-tile slots
+  int n_units, n_qb;  // units: n_qb query blocks x (up to) tpu-tile slots
+  int tpu;            // key tiles per unit: kTilesPerUnit, or fewer when that leaves SMs idle
   WsHeader* ws;
 };
 
@@ -102,8 +103,8 @@ __device__ __forceinline__ bool unit_range(const IdxParams& p, int u, int& qb, i
   qb = p.n_qb - 1 - (u - c * p.n_qb);
   const int last_q = min((qb + 1) * C::kQB, p.n_q) - 1;
   const int ntiles = (p.q_pos0 + last_q) / C::kM + 1;
-  kt0 = c * C::kTilesPerUnit;
-  kt1 = min(kt0 + C::kTilesPerUnit, ntiles);
+  kt0 = c * p.tpu;
+  kt1 = min(kt0 + p.tpu, ntiles);
   return kt0 < kt1;
 }
 
@@ -407,8 +408,15 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_i
   p.q_pos0 = d.q_pos0;
   p.ws = ws;
   const int max_tiles = (d.q_pos0 + d.n_q - 1) / C::kM + 1;
-  const int slots = (max_tiles + C::kTilesPerUnit - 1) / C::kTilesPerUnit;
   p.n_qb = (d.n_q + C::kQB - 1) / C::kQB;
+  // 32 tiles per unit, or fewer when a small chunk (a decode step) would then
+  // give fewer units than SMs; a score does not depend on the unit it is in
+  p.tpu = C::kTilesPerUnit;
+  const long long tiles_total = static_cast<long long>(p.n_qb) * max_tiles;
+  if (tiles_total < static_cast<long long>(C::kTilesPerUnit) * num_sms())
+    p.tpu = static_cast<int>((tiles_total + num_sms() - 1) / num_sms());
+  if (p.tpu < 1) p.tpu = 1;
+  const int slots = (max_tiles + p.tpu - 1) / p.tpu;
   p.n_units = p.n_qb * slots;
   // the work queue starts at unit 0 on every launch
   cudaError_t e0 = cudaMemsetAsync(&ws->unit_next, 0, sizeof(ws->unit_next), st);

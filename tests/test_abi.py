@@ -73,6 +73,13 @@ def test_workspace_sizes(dsa):
     ld = (d.ctx_len + 127) // 128 * 128
     assert dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER) == 256 + d.n_q * ld * 4 + d.n_q * d.top_k * 4
     assert dsa.dsa_workspace_size(d, 99) == 0
+    # decode: the split attention's partials (n_split ranges of H x (Dc + 2) floats per query)
+    d1 = workloads.make_dims(1, 49151, 49152, 32, 512, 64, 32, 128, 2048)
+    part = 16 * 32 * 512 * 4 + (16 * 32 * 8 + 255) // 256 * 256  # 148 SMs: n_split = 16
+    assert dsa.dsa_workspace_size(d1, dsa.DSA_WS_DECODE_ATTN) == 256 + part
+    ld1 = 49152
+    layer1 = 256 + ld1 * 4 + (2048 * 4 + 255) // 256 * 256
+    assert dsa.dsa_workspace_size(d1, dsa.DSA_WS_DECODE_LAYER) == layer1 + part
 
 
 FAKE = 1 << 20  # an aligned, never dereferenced address
