@@ -62,8 +62,9 @@ def _load():
         lib.oracle_topk_select_f32.argtypes = [dp, P, i64, P, i32, P, cint]
         lib.oracle_sparse_attn.argtypes = [dp, P, P, P, P, P, i32, P, P, cint]
         lib.oracle_prefill_layer.argtypes = [dp, P, P, P, P, P, P, P, i32, P, P, P, cint]
+        lib.oracle_quantize_fp8.argtypes = [P, i64, i32, P, P, P]
         for f in (lib.oracle_index_scores, lib.oracle_topk_select, lib.oracle_topk_select_f32,
-                  lib.oracle_sparse_attn, lib.oracle_prefill_layer):
+                  lib.oracle_sparse_attn, lib.oracle_prefill_layer, lib.oracle_quantize_fp8):
             f.restype = cint
         _lib = lib
     return _lib
@@ -162,3 +163,26 @@ def prefill_layer(d, q, latent, rope, q_idx, k_idx, w_idx, rows=None, n_threads=
                                       _ptr(out), _ptr(lse), _ptr(idx), _threads(n_threads))
     assert rc == 0
     return out, lse, idx
+
+
+def quantize_fp8(x):
+    """FP8 (e4m3) form of bf16 rows x [..., cols] (see dsa_oracle.cpp):
+    (x8 uint8 e4m3 bits, scale float32 [...], xhat uint16 bf16 bits)."""
+    x = _u16(x)
+    shape = x.shape
+    cols = shape[-1]
+    rows = int(np.prod(shape[:-1])) if len(shape) > 1 else 1
+    x8 = np.empty(shape, dtype=np.uint8)
+    scale = np.empty(shape[:-1], dtype=np.float32)
+    xhat = np.empty(shape, dtype=np.uint16)
+    rc = _load().oracle_quantize_fp8(_ptr(x), rows, cols, _ptr(x8), _ptr(scale), _ptr(xhat))
+    assert rc == 0
+    return x8, scale, xhat
+
+
+def index_scores_fp8(d, q_idx, k_idx, w_idx, rows=None, n_threads=None):
+    """Scores of the FP8 indexer contract: the float64 scores of the
+    dequantized (xhat) indexer inputs."""
+    _, _, q_hat = quantize_fp8(q_idx)
+    _, _, k_hat = quantize_fp8(k_idx)
+    return index_scores(d, q_hat, k_hat, w_idx, rows=rows, n_threads=n_threads)

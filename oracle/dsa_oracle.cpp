@@ -247,6 +247,63 @@ int oracle_sparse_attn(const oracle_dims* d, const uint16_t* q, const uint16_t* 
   return 0;
 }
 
+// FP8 (e4m3) form of indexer inputs, for the FP8 indexer variant. The pages do
+// not describe one; this follows the layer's published design in spirit (an
+// 8-bit indexer) with the plainest exact rules:
+//   scale  the smallest power of two s = 2^k with max_c |x[r,c]| <= 448 s
+//          (448 is the largest finite e4m3 value; s = 1 for an all-zero row);
+//   x8     x / s rounded to the nearest e4m3 value, ties to even: 4
+//          significant bits for |x/s| >= 2^-6, multiples of 2^-9 below
+//          (subnormals); the sign is kept, also on a zero;
+//   xhat   x8 * s, the dequantized value (exact, and a bf16 value).
+// The FP8 indexer's score contract is the bf16 contract (index_score) applied
+// to the dequantized rows xhat.
+// x: bf16 [rows, cols]; x8: e4m3 bit patterns [rows, cols]; scale: float
+// [rows]; xhat: bf16 [rows, cols].
+int oracle_quantize_fp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* x8, float* scale,
+                        uint16_t* xhat) {
+  if (!x || !x8 || !scale || !xhat || rows < 0 || cols < 1) return -1;
+  for (int64_t r = 0; r < rows; ++r) {
+    const uint16_t* xr = x + r * cols;
+    double amax = 0.0;
+    for (int c = 0; c < cols; ++c) amax = std::max(amax, std::fabs(bf16_to_double(xr[c])));
+    int k = 0;
+    if (amax > 0.0) {
+      k = std::ilogb(amax) - 9;  // 448 * 2^k < amax here; step up to the first k that covers it
+      while (amax > std::ldexp(448.0, k)) ++k;
+    }
+    scale[r] = static_cast<float>(std::ldexp(1.0, k));
+    for (int c = 0; c < cols; ++c) {
+      const double xv = bf16_to_double(xr[c]);
+      const double v = std::ldexp(xv, -k);  // exact
+      const double av = std::fabs(v);
+      double qv = 0.0;  // |x8| as a value
+      if (av > 0.0) {
+        const int e = std::ilogb(av);
+        const double quantum = e < -6 ? std::ldexp(1.0, -9) : std::ldexp(1.0, e - 3);
+        qv = std::nearbyint(av / quantum) * quantum;  // round half to even
+      }
+      uint8_t bits = std::signbit(v) ? 0x80 : 0x00;
+      if (qv > 0.0) {
+        const int e2 = std::ilogb(qv);
+        if (e2 < -6) {
+          bits |= static_cast<uint8_t>(qv / std::ldexp(1.0, -9));           // subnormal: m * 2^-9
+        } else {
+          const int mant = static_cast<int>(qv / std::ldexp(1.0, e2 - 3)) - 8;  // 1.mmm * 2^e2
+          bits |= static_cast<uint8_t>(((e2 + 7) << 3) | mant);
+        }
+      }
+      x8[r * cols + c] = bits;
+      const double hat = std::signbit(v) ? -std::ldexp(qv, k) : std::ldexp(qv, k);
+      const float hf = static_cast<float>(hat);  // exact: 4 significant bits
+      uint32_t hb;
+      std::memcpy(&hb, &hf, sizeof hb);
+      xhat[r * cols + c] = static_cast<uint16_t>(hb >> 16);
+    }
+  }
+  return 0;
+}
+
 // The whole layer for the listed query rows: scores -> selection -> attention.
 // idx_out ([n_rows, k]) and lse ([n_rows, H]) may be null.
 int oracle_prefill_layer(const oracle_dims* d, const uint16_t* q, const uint16_t* latent,

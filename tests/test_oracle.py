@@ -366,3 +366,59 @@ def test_stored_selection_digests_match_the_oracle():
             sel = mod.oracle_selection(d, x, rows=rows)
             _, digests = mod.selection_digests(sel)
             assert digests[0] == c["block_sha256"][b], (key, b)
+
+
+# ------------------------------------------------ FP8 form of the indexer inputs
+
+
+def test_fp8_hand_case(oracle_lib):
+    with open(os.path.join(GOLDEN, "fp8_hand_case.json")) as f:
+        g = json.load(f)
+    x = _bf16([g["x"]])
+    x8, scale, xhat = oracle_lib.quantize_fp8(x)
+    assert float(scale[0]) == g["expected_scale"]
+    assert x8[0].tolist() == g["expected_codes"]
+    assert bf16_bits_to_f32(xhat)[0].tolist() == g["expected_xhat"]
+
+
+def test_fp8_codes_match_torch_e4m3_conversion(oracle_lib):
+    """e4m3 codes against torch's float8_e4m3fn conversion of x / scale (round
+    to nearest even), on normal draws, small values (subnormal codes), zeros of
+    both signs and an all-zero row; the scale is the smallest power of two that
+    covers the row's maximum."""
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((64, 128)).astype(np.float32)
+    x[3] *= 1e-3
+    x[4, :64] *= 1e-4                # subnormal e4m3 codes after scaling
+    x[5] = 0.0
+    x[6, ::3] = -0.0
+    x[7] = np.round(x[7] * 8) / 8    # many ties
+    xb = _bf16(x)
+    x8, scale, xhat = oracle_lib.quantize_fp8(xb)
+    xf = bf16_bits_to_f32(xb).astype(np.float64)
+    amax = np.abs(xf).max(axis=1)
+    s = scale.astype(np.float64)
+    assert np.all(np.log2(s) == np.round(np.log2(s)))          # powers of two
+    nz = amax > 0
+    assert np.all(amax[nz] <= 448 * s[nz]) and np.all(amax[nz] > 224 * s[nz])
+    assert np.all(s[~nz] == 1.0)
+    ref = torch.from_numpy((xf / s[:, None]).astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(x8, ref.view(torch.uint8).numpy())
+    deq = ref.to(torch.float64).numpy() * s[:, None]
+    assert np.array_equal(bf16_bits_to_f32(xhat).astype(np.float64), deq)
+
+
+def test_fp8_contract_scores_match_torch_on_dequantized_inputs(oracle_lib):
+    d, x = _small_inputs(seed=13)
+    sc = oracle_lib.index_scores_fp8(d, x["q_idx"], x["k_idx"], x["w_idx"])
+    _, _, qh = oracle_lib.quantize_fp8(x["q_idx"])
+    _, _, kh = oracle_lib.quantize_fp8(x["k_idx"])
+    qi, ki = torch.from_numpy(_f64(qh)), torch.from_numpy(_f64(kh))
+    w = torch.from_numpy(x["w_idx"].astype(np.float64))
+    ref = torch.einsum("nj,njs->ns", w, torch.relu(torch.einsum("njc,sc->njs", qi, ki))).numpy()
+    t = d.q_pos0 + np.arange(d.n_q)[:, None]
+    causal = np.arange(d.ctx_len)[None, :] <= t
+    np.testing.assert_allclose(sc[causal], ref[causal], rtol=1e-13, atol=1e-13)
+    # the 8-bit form moves scores, but not far: within a few percent of the bf16 scores
+    sb = oracle_lib.index_scores(d, x["q_idx"], x["k_idx"], x["w_idx"])
+    assert np.abs(sc[causal] - sb[causal]).max() <= 0.1 * np.abs(sb[causal]).max()
