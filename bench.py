@@ -23,6 +23,7 @@ the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -48,6 +49,7 @@ L2_FLUSH_BYTES = 256 << 20
 PROFILED_DRAM_BYTES_PER_LAUNCH: dict = {}
 
 KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
+# (the FP8 indexer variant adds the e4m3 forms of the keys and of the queries)
 E2E_SUB_CHUNKS = (8, 16, 32, 64)  # query sub-chunk counts tried for the host-buffer call (copies overlap the layer)
 
 
@@ -238,6 +240,42 @@ def time_steps(step, flush, steps, stream, flushed=True):
     return [a.elapsed_time(b) for a, b in zip(starts, ends)]
 
 
+def attn_variants(dsa, d, xd, idx, out, lse, flush, stream, steps):
+    """Median CUDA-event time (ms) of the attention step alone in each of its
+    forms on the layer's own selection: the per-query pipelined kernel, the
+    decode split and the block-sparse union over groups of 1 and 2 queries."""
+    import torch
+
+    ws = {}
+
+    def ws_for(which):
+        if which not in ws:
+            ws[which] = torch.empty(max(256, dsa.dsa_workspace_size(d, which)), dtype=torch.uint8,
+                                    device="cuda")
+        return ws[which]
+
+    calls = {
+        "per_query": lambda: dsa.dsa_sparse_attn_prefill(
+            d, xd["q"], xd["latent"], xd["rope"], idx, out, lse, ws_for(dsa.DSA_WS_ATTN),
+            stream=stream),
+        "decode_split": lambda: dsa.dsa_sparse_attn_decode(
+            d, xd["q"], xd["latent"], xd["rope"], idx, out, lse, ws_for(dsa.DSA_WS_DECODE_ATTN),
+            stream=stream),
+        "block_qb1": lambda: dsa.dsa_sparse_attn_block(
+            d, xd["q"], xd["latent"], xd["rope"], idx, out, lse, 1, ws_for(dsa.DSA_WS_BLOCK_ATTN),
+            stream=stream),
+        "block_qb2": lambda: dsa.dsa_sparse_attn_block(
+            d, xd["q"], xd["latent"], xd["rope"], idx, out, lse, 2, ws_for(dsa.DSA_WS_BLOCK_ATTN),
+            stream=stream),
+    }
+    res = {}
+    for name, call in calls.items():
+        dsa.check(call())  # warm-up
+        res[name] = statistics.median(
+            time_steps(lambda: dsa.check(call()), flush, max(3, steps), stream))
+    return res
+
+
 def run_ours(args):
     import torch
 
@@ -258,6 +296,10 @@ def run_ours(args):
     d = wl.dims
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     x = workloads.generate(d, rank_seed(wl.seed, rank), wl.kind, w_mode)
+    if args.fp8_indexer:  # the FP8 indexer variant of the layer (its own selection contract)
+        import dataclasses
+
+        d = dataclasses.replace(d, flags=dsa.DSA_FLAG_FP8_INDEXER)
     stream = torch.cuda.current_stream()
 
     def to_dev_bf16(a):
@@ -314,21 +356,41 @@ def run_ours(args):
 
     # ---- per-kernel durations, same inputs and launch configuration
     ld = (d.ctx_len + 127) // 128 * 128
-    scores = ws_layer[256:256 + d.n_q * ld * 4].view(torch.float32).view(d.n_q, ld)
+    scores = torch.empty(d.n_q, ld, dtype=torch.float32, device="cuda")
     ws_small = torch.empty(256, dtype=torch.uint8, device="cuda")
     names = ("index_scores", "topk_select", "sparse_attn")
+    d1 = dataclasses.replace(d, flags=0)  # the single-step calls take no flag
+    if args.fp8_indexer:
+        # the e4m3 keys are formed once per cache (as in the layer); the
+        # queries' e4m3 form is part of the timed indexer step
+        q_rows = d.n_q * d.n_idx_heads
+        k8 = torch.empty(d.ctx_len, d.d_idx, dtype=torch.uint8, device="cuda")
+        ks = torch.empty(d.ctx_len, dtype=torch.float32, device="cuda")
+        kh = torch.empty(d.ctx_len, d.d_idx, dtype=torch.int16, device="cuda")
+        q8 = torch.empty(q_rows, d.d_idx, dtype=torch.uint8, device="cuda")
+        qs = torch.empty(q_rows, dtype=torch.float32, device="cuda")
+        qh = torch.empty(q_rows, d.d_idx, dtype=torch.int16, device="cuda")
+        dsa.check(dsa.dsa_quantize_fp8(xd["k_idx"], d.ctx_len, d.d_idx, k8, ks, kh, stream=stream))
+        q_in, k_in = qh, kh
+    else:
+        q_in, k_in = xd["q_idx"], xd["k_idx"]
     ev = []
     for s in range(args.steps):
         flush.zero_()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         e[0].record(stream)
-        dsa.check(dsa.dsa_index_scores(d, xd["q_idx"], xd["k_idx"], xd["w_idx"], scores, ld,
-                                       ws_small, stream=stream))
+        if args.fp8_indexer:
+            dsa.check(dsa.dsa_quantize_fp8(xd["q_idx"], q_rows, d.d_idx, q8, qs, qh, stream=stream))
+            dsa.check(dsa.dsa_index_scores_fp8(d1, q8, qs, k8, ks, xd["w_idx"], scores, ld,
+                                               ws_small, stream=stream))
+        else:
+            dsa.check(dsa.dsa_index_scores(d1, xd["q_idx"], xd["k_idx"], xd["w_idx"], scores, ld,
+                                           ws_small, stream=stream))
         e[1].record(stream)
-        dsa.check(dsa.dsa_topk_select(d, scores, ld, xd["q_idx"], xd["k_idx"], xd["w_idx"], idx,
+        dsa.check(dsa.dsa_topk_select(d1, scores, ld, q_in, k_in, xd["w_idx"], idx,
                                       ws_small, stream=stream))
         e[2].record(stream)
-        dsa.check(dsa.dsa_sparse_attn_prefill(d, xd["q"], xd["latent"], xd["rope"], idx, out,
+        dsa.check(dsa.dsa_sparse_attn_prefill(d1, xd["q"], xd["latent"], xd["rope"], idx, out,
                                               lse, ws_small, stream=stream))
         e[3].record(stream)
         ev.append(e)
@@ -336,6 +398,8 @@ def run_ours(args):
     per_kernel = {n: statistics.median(e[j].elapsed_time(e[j + 1]) for e in ev)
                   for j, n in enumerate(names)}
     rates = kernel_rates(d, per_kernel, peaks)
+    variants = attn_variants(dsa, d1, xd, idx, out, lse, flush, stream, args.steps) \
+        if args.attn_variants else None
 
     # ---- end to end through the library's host-buffer call: every step copies
     # all inputs in from page-locked host memory and the output back, the
@@ -416,6 +480,7 @@ def run_ours(args):
                    "ctx_len": d.ctx_len, "top_k": d.top_k, "n_heads": d.n_heads,
                    "d_latent": d.d_latent, "d_rope": d.d_rope, "n_idx_heads": d.n_idx_heads,
                    "d_idx": d.d_idx, "parallelism": f"dp{world} (independent chunks)",
+                   "indexer": "fp8 (e4m3) variant" if args.fp8_indexer else "bf16",
                    "l2": "flushed: 256 MB write between timed steps"},
         "tflops": tflops,
         "pct_of_measured_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
@@ -425,12 +490,13 @@ def run_ours(args):
         "warm_l2": {"ms_per_step_median": warm_ms_per_step,
                     "value": whole_job_rate(world, d.n_q, warm_ms_per_step)},
         "per_kernel_ms": per_kernel,
+        **({"attn_variants_ms": variants} if variants else {}),
         "per_kernel": rates,
         "e2e": {"value": whole_job_rate(world, d.n_q, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "call": "dsa_prefill_layer_host", "sub_chunks": n_best,
                 "warmup_ms_by_sub_chunks": {str(k): round(v, 3) for k, v in tried.items()}},
-        "gpu_launches": KERNELS_PER_LAYER * args.steps,
+        "gpu_launches": (KERNELS_PER_LAYER + (2 if args.fp8_indexer else 0)) * args.steps,
         "roofline": roof,
         "clocks": clocks.summary(),
     }
@@ -641,6 +707,10 @@ def main():
     ap.add_argument("--split", default="chunks", choices=("chunks", "query"),
                     help="chunks: every rank runs its own chunk (weak scaling, default); "
                          "query: one chunk split by queries over the ranks (strong scaling)")
+    ap.add_argument("--attn-variants", action="store_true",
+                    help="also time the attention step's other forms (decode split, block union)")
+    ap.add_argument("--fp8-indexer", action="store_true",
+                    help="the layer with the FP8 indexer variant (dims.flags = DSA_FLAG_FP8_INDEXER)")
     ap.add_argument("--layer-only", action="store_true",
                     help="time the layer alone and print a short line (for profiler captures)")
     args = ap.parse_args()

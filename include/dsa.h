@@ -56,8 +56,16 @@ typedef struct dsa_dims {
   int32_t d_idx;       /* indexer head width D_I                                      */
   int32_t top_k;       /* keys kept per query, 1..DSA_MAX_TOPK                        */
   float softmax_scale; /* multiplies the attention logits                             */
-  uint32_t flags;      /* must be 0                                                   */
+  uint32_t flags;      /* 0, or DSA_FLAG_FP8_INDEXER in the whole-layer calls         */
 } dsa_dims;
+
+/* dims.flags: the whole-layer calls (dsa_prefill_layer, dsa_decode_layer,
+ * dsa_prefill_layer_host, dsa_prefill_layer_noalloc) score with the FP8
+ * indexer: q_idx and k_idx are taken to their e4m3 form (dsa_quantize_fp8,
+ * in the workspace), scored by dsa_index_scores_fp8, and the exact top-k
+ * orders keys by the float64 contract of dsa_topk_select on the dequantized
+ * rows. Every other call requires flags == 0. */
+#define DSA_FLAG_FP8_INDEXER 1u
 
 /* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):
  *   (n_heads, d_latent, d_rope)  in {(4, 64, 16), (32, 512, 64)}
@@ -87,6 +95,7 @@ typedef int32_t dsa_status;
 #define DSA_WS_LAYER 3
 #define DSA_WS_DECODE_ATTN 4
 #define DSA_WS_DECODE_LAYER 5
+#define DSA_WS_BLOCK_ATTN 6
 
 /* Bytes of device workspace the call `which` needs for these dims (0 on bad
  * arguments). The first 256 bytes of every workspace hold the device status
@@ -110,6 +119,37 @@ size_t dsa_workspace_size(const dsa_dims* dims, int32_t which);
 dsa_status dsa_index_scores(const dsa_dims* dims, const uint16_t* q_idx, const uint16_t* k_idx,
                             const float* w_idx, float* scores, int64_t ld_scores,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* FP8 (e4m3) form of bf16 rows for the FP8 indexer (an 8-bit form of the
+ * "DSA indexer" row of the feedman.me post's component table; the pages
+ * describe no FP8 indexer, these are this library's rules). For each of the
+ * `rows` rows of `cols` (1..128) values:
+ *   scale[r] = the smallest power of two s with max_c |x[r,c]| <= 448 s
+ *              (1 for an all-zero row; 448 is the largest finite e4m3 value);
+ *   x8[r,c]  = x[r,c] / s rounded to the nearest e4m3 value, ties to even
+ *              (the bit pattern; the sign of a zero is kept);
+ *   xhat[r,c]= x8[r,c] * s as bf16 (exact).
+ *   x     bf16 [rows, cols]     x8    uint8 [rows, cols]
+ *   scale f32  [rows]           xhat  bf16  [rows, cols]
+ * Indexer rows are k_idx [ctx_len, d_idx] and q_idx [n_q * n_idx_heads,
+ * d_idx]. Errors: DSA_ERR_DIMS, _NULL, _ALIGN, _DEVICE, _CUDA. */
+dsa_status dsa_quantize_fp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* x8,
+                            float* scale, uint16_t* xhat, void* stream);
+
+/* Lightning-indexer scores from e4m3 operands (tensor cores, kind::f8f6f4,
+ * float32 accumulation): for s <= t,
+ *     I[i,s] = s_k[s] * sum_j w_idx[i,j] * s_q[i,j] * ReLU( sum_c q8[i,j,c] * k8[s,c] )
+ * which is the score of dsa_index_scores on the dequantized rows (xhat) up to
+ * float32 rounding, within the same error bound, so dsa_topk_select given the
+ * dequantized rows orders these scores exactly.
+ *   q8 uint8 [n_q, n_idx_heads, d_idx], q_scale f32 [n_q, n_idx_heads],
+ *   k8 uint8 [ctx_len, d_idx], k_scale f32 [ctx_len] (from dsa_quantize_fp8);
+ *   w_idx, scores, ld_scores and the workspace as in dsa_index_scores.
+ * Errors: those of dsa_index_scores. */
+dsa_status dsa_index_scores_fp8(const dsa_dims* dims, const uint8_t* q8, const float* q_scale,
+                                const uint8_t* k8, const float* k_scale, const float* w_idx,
+                                float* scores, int64_t ld_scores, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Per-query top-k selection (the "per-query top-2048" step of the feedman.me
  * post, paragraph after the component table). Among s = 0..t, keys are
@@ -194,6 +234,29 @@ dsa_status dsa_decode_layer(const dsa_dims* dims, const uint16_t* q, const uint1
                             const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                             const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention (the feedman.me post's proposed fix, paragraph "Two
+ * levers fell out of this": share gathered keys across neighbouring queries
+ * and use the matrix units). Queries are taken in groups of block_queries
+ * (1 or 2) neighbours; each group gathers the union of its queries' selected
+ * keys once, in ascending key order, and runs QK^T and PV for all of the
+ * group's heads on it, a key outside a query's own selection being masked
+ * (p = 0) for that query. Same definition, arguments, layouts and errors as
+ * dsa_sparse_attn_prefill, with each valid key listed at most once per idx
+ * row (as every selection is); entries past t are reported as DSA_ERR_RANGE
+ * and skipped. Workspace: dsa_workspace_size(dims, DSA_WS_BLOCK_ATTN) bytes
+ * (the union lists and masks). block_queries = 1 runs the same kernel per
+ * query. This kernel runs its steps one after another (a tile of the union
+ * and the group's q rows fill shared memory); dsa_sparse_attn_prefill, which
+ * pipelines the gather under the tensor-core work, is the faster path on the
+ * measured workloads, and this call exists to measure the union against it.
+ * Errors: those of dsa_sparse_attn_prefill, DSA_ERR_DIMS for block_queries
+ * outside 1..DSA_MAX_BLOCK_QUERIES. */
+#define DSA_MAX_BLOCK_QUERIES 2
+dsa_status dsa_sparse_attn_block(const dsa_dims* dims, const uint16_t* q, const uint16_t* latent,
+                                 const uint16_t* rope, const int32_t* idx, uint16_t* out,
+                                 float* lse, int32_t block_queries, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Device copies of the layer's tensors for dsa_prefill_layer_host, owned by
  * the caller, each of the full size given under dsa_prefill_layer and 16-byte

@@ -44,6 +44,9 @@ DSA_WS_ATTN = 2
 DSA_WS_LAYER = 3
 DSA_WS_DECODE_ATTN = 4
 DSA_WS_DECODE_LAYER = 5
+DSA_WS_BLOCK_ATTN = 6
+DSA_FLAG_FP8_INDEXER = 1
+DSA_MAX_BLOCK_QUERIES = 2
 
 DSA_MAX_TOPK = 2048
 DSA_MAX_CTX = 49152
@@ -52,7 +55,8 @@ EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",
             "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host",
             "dsa_selftest_bounded_wait", "dsa_partition_queries", "dsa_sparse_attn_decode",
-            "dsa_decode_layer")
+            "dsa_decode_layer", "dsa_sparse_attn_block", "dsa_quantize_fp8",
+            "dsa_index_scores_fp8")
 
 
 class dsa_dims(ctypes.Structure):
@@ -107,6 +111,11 @@ def library():
     lib.dsa_sparse_attn_decode.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     lib.dsa_decode_layer.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]
+    lib.dsa_sparse_attn_block.argtypes = [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P,
+                                          ctypes.c_size_t, _P]
+    lib.dsa_quantize_fp8.argtypes = [_P, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P]
+    lib.dsa_index_scores_fp8.argtypes = [_DP, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
+                                         ctypes.c_size_t, _P]
     lib.dsa_prefill_layer_noalloc.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
     lib.dsa_prefill_layer_host.argtypes = [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
@@ -119,7 +128,8 @@ def library():
     for f in ("dsa_index_scores", "dsa_topk_select", "dsa_sparse_attn_prefill",
               "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc",
               "dsa_prefill_layer_host", "dsa_selftest_bounded_wait", "dsa_partition_queries",
-              "dsa_sparse_attn_decode", "dsa_decode_layer"):
+              "dsa_sparse_attn_decode", "dsa_decode_layer", "dsa_sparse_attn_block",
+              "dsa_quantize_fp8", "dsa_index_scores_fp8"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -199,6 +209,25 @@ def dsa_sparse_attn_decode(dims, q, latent, rope, idx, out, lse, workspace, work
     return library().dsa_sparse_attn_decode(_dims(dims), _p(q), _p(latent), _p(rope), _p(idx),
                                             _p(out), _p(lse), _p(workspace),
                                             _nbytes(workspace, workspace_bytes), _stream(stream))
+
+
+def dsa_sparse_attn_block(dims, q, latent, rope, idx, out, lse, block_queries, workspace,
+                          workspace_bytes=None, stream=None) -> int:
+    return library().dsa_sparse_attn_block(_dims(dims), _p(q), _p(latent), _p(rope), _p(idx),
+                                           _p(out), _p(lse), int(block_queries), _p(workspace),
+                                           _nbytes(workspace, workspace_bytes), _stream(stream))
+
+
+def dsa_quantize_fp8(x, rows, cols, x8, scale, xhat, stream=None) -> int:
+    return library().dsa_quantize_fp8(_p(x), int(rows), int(cols), _p(x8), _p(scale), _p(xhat),
+                                      _stream(stream))
+
+
+def dsa_index_scores_fp8(dims, q8, q_scale, k8, k_scale, w_idx, scores, ld_scores, workspace,
+                         workspace_bytes=None, stream=None) -> int:
+    return library().dsa_index_scores_fp8(_dims(dims), _p(q8), _p(q_scale), _p(k8), _p(k_scale),
+                                          _p(w_idx), _p(scores), int(ld_scores), _p(workspace),
+                                          _nbytes(workspace, workspace_bytes), _stream(stream))
 
 
 def dsa_decode_layer(dims, q, latent, rope, q_idx, k_idx, w_idx, out, lse, idx_out, workspace,

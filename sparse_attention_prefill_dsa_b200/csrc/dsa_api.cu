@@ -52,9 +52,10 @@ bool indexer_shape_ok(const dsa_dims& d) {
 
 // Common shape checks. `need_attn` / `need_indexer` select which head shapes
 // the call uses.
-dsa_status check_dims(const dsa_dims* d, bool need_attn, bool need_indexer) {
+dsa_status check_dims(const dsa_dims* d, bool need_attn, bool need_indexer,
+                      uint32_t allowed_flags = 0u) {
   if (!d) return DSA_ERR_NULL;
-  if (d->flags != 0u) return DSA_ERR_DIMS;
+  if ((d->flags & ~allowed_flags) != 0u) return DSA_ERR_DIMS;
   if (d->n_q < 0 || d->q_pos0 < 0 || d->ctx_len < 1 || d->ctx_len > DSA_MAX_CTX)
     return DSA_ERR_DIMS;
   if (d->top_k < 1 || d->top_k > DSA_MAX_TOPK) return DSA_ERR_DIMS;
@@ -71,21 +72,59 @@ size_t layer_scores_bytes(const dsa_dims& d) {
   return static_cast<size_t>(d.n_q) * layer_ld(d) * sizeof(float);
 }
 
-int32_t* layer_idx_region(void* ws, const dsa_dims& d) {
-  return reinterpret_cast<int32_t*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes +
-                                    layer_scores_bytes(d));
-}
 
-size_t layer_bytes(const dsa_dims& d) {
-  return dsa::kWsHeaderBytes + layer_scores_bytes(d) +
-         (static_cast<size_t>(d.n_q) * d.top_k * sizeof(int32_t) + 255) / 256 * 256;
+size_t r256(size_t b) { return (b + 255) / 256 * 256; }
+
+bool fp8_indexer(const dsa_dims& d) { return (d.flags & DSA_FLAG_FP8_INDEXER) != 0u; }
+
+// e4m3 codes, scales and dequantized bf16 copies of `rows` rows of `cols`
+size_t fp8_rows_bytes(size_t rows, int cols) {
+  return r256(rows * cols) + r256(rows * 4) + r256(rows * cols * 2);
 }
 
 // decode: the split attention's partials follow the header (attention alone)
-// or the layer's score and selection regions (whole layer)
+// or the layer's other regions (whole layer)
 size_t decode_part_bytes(const dsa_dims& d) {
   const int n_split = dsa::attn_decode_split(d);
   return n_split > 1 ? dsa::attn_split_bytes(d.n_q, n_split, d.n_heads, d.d_latent) : 0;
+}
+
+// Byte offsets of the layer's workspace regions: the header; with the FP8
+// indexer the keys' e4m3 form (it depends on the cache only, so sub-chunks of
+// one chunk find it at the same place); the float32 scores; the selection;
+// with the FP8 indexer the queries' e4m3 form; for decode the split
+// attention's partials. Without either option this is header | scores | idx.
+struct LayerWs {
+  size_t kfp8, scores, idx, qfp8, part, total;
+};
+
+LayerWs layer_ws(const dsa_dims& d, bool decode) {
+  const bool f8 = fp8_indexer(d);
+  const size_t idx_bytes = static_cast<size_t>(d.n_q) * d.top_k * sizeof(int32_t);
+  LayerWs w;
+  w.kfp8 = dsa::kWsHeaderBytes;
+  w.scores = w.kfp8 + (f8 ? fp8_rows_bytes(static_cast<size_t>(d.ctx_len), d.d_idx) : 0);
+  w.idx = w.scores + layer_scores_bytes(d);
+  w.qfp8 = w.idx + (f8 || decode ? r256(idx_bytes) : idx_bytes);
+  w.part = w.qfp8 + (f8 ? fp8_rows_bytes(static_cast<size_t>(d.n_q) * d.n_idx_heads, d.d_idx) : 0);
+  w.total = w.part + (decode ? decode_part_bytes(d) : 0);
+  return w;
+}
+
+// Pointers of one FP8 region (codes, scales, dequantized rows) at byte `off`.
+struct Fp8Rows {
+  uint8_t* x8;
+  float* scale;
+  uint16_t* xhat;
+};
+
+Fp8Rows fp8_rows(void* ws, size_t off, size_t rows, int cols) {
+  char* b = static_cast<char*>(ws) + off;
+  Fp8Rows r;
+  r.x8 = reinterpret_cast<uint8_t*>(b);
+  r.scale = reinterpret_cast<float*>(b + r256(rows * cols));
+  r.xhat = reinterpret_cast<uint16_t*>(b + r256(rows * cols) + r256(rows * 4));
+  return r;
 }
 
 dsa_status check_ws(const dsa_dims& d, int which, void* ws, size_t bytes) {
@@ -113,23 +152,44 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
                          cudaStream_t st, bool norms_ready = false, bool decode = false) {
   if (d.n_q == 0) return DSA_OK;
   WsHeader* h = static_cast<WsHeader*>(ws);
-  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + dsa::kWsHeaderBytes);
+  const LayerWs w = layer_ws(d, decode);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + w.scores);
   const int64_t ld = layer_ld(d);
   // The selection goes to the caller's idx_out when given, else to the
   // workspace region after the score matrix.
-  int32_t* idx = idx_out ? idx_out : layer_idx_region(ws, d);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.idx);
   cudaError_t e = cudaSuccess;
-  if (!norms_ready) {
-    e = dsa::launch_key_norm_max(d, k_idx, h, st);
-    if (e == cudaSuccess) e = dsa::launch_attn_key_norm_max(d, latent, rope, h, st);
+  if (fp8_indexer(d)) {
+    // FP8 indexer: the e4m3 forms of k_idx (once per cache) and q_idx; the
+    // exact top-k orders by the float64 contract on their dequantized rows
+    const Fp8Rows k8 = fp8_rows(ws, w.kfp8, static_cast<size_t>(d.ctx_len), d.d_idx);
+    const size_t q_rows = static_cast<size_t>(d.n_q) * d.n_idx_heads;
+    const Fp8Rows q8 = fp8_rows(ws, w.qfp8, q_rows, d.d_idx);
+    if (!norms_ready) {
+      e = dsa::launch_quantize_fp8(k_idx, d.ctx_len, d.d_idx, k8.x8, k8.scale, k8.xhat, st);
+      if (e == cudaSuccess) e = dsa::launch_key_norm_max(d, k8.xhat, h, st);
+      if (e == cudaSuccess) e = dsa::launch_attn_key_norm_max(d, latent, rope, h, st);
+    }
+    if (e == cudaSuccess)
+      e = dsa::launch_quantize_fp8(q_idx, static_cast<int64_t>(q_rows), d.d_idx, q8.x8, q8.scale,
+                                   q8.xhat, st);
+    if (e == cudaSuccess)
+      e = dsa::launch_index_scores_fp8(d, q8.x8, q8.scale, k8.x8, k8.scale, w_idx, scores, ld, h, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    e = dsa::launch_topk(d, scores, ld, q8.xhat, k8.xhat, w_idx, idx, h, st);
+  } else {
+    if (!norms_ready) {
+      e = dsa::launch_key_norm_max(d, k_idx, h, st);
+      if (e == cudaSuccess) e = dsa::launch_attn_key_norm_max(d, latent, rope, h, st);
+    }
+    if (e == cudaSuccess) e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
   }
-  if (e == cudaSuccess) e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
-  if (e != cudaSuccess) return DSA_ERR_CUDA;
-  e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (decode) {
     const int n_split = dsa::attn_decode_split(d);
-    void* part = n_split > 1 ? static_cast<char*>(ws) + layer_bytes(d) : nullptr;
+    void* part = n_split > 1 ? static_cast<char*>(ws) + w.part : nullptr;
     return from_cuda(
         dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, true, h, st, n_split, part));
   }
@@ -156,12 +216,13 @@ size_t dsa_workspace_size(const dsa_dims* d, int32_t which) {
     case DSA_WS_ATTN:
       return dsa::kWsHeaderBytes;
     case DSA_WS_LAYER:
-      return dsa::kWsHeaderBytes + layer_scores_bytes(*d) +
-             static_cast<size_t>(d->n_q) * d->top_k * sizeof(int32_t);
+      return layer_ws(*d, false).total;
     case DSA_WS_DECODE_ATTN:
       return dsa::kWsHeaderBytes + decode_part_bytes(*d);
     case DSA_WS_DECODE_LAYER:
-      return layer_bytes(*d) + decode_part_bytes(*d);
+      return layer_ws(*d, true).total;
+    case DSA_WS_BLOCK_ATTN:
+      return dsa::kWsHeaderBytes + dsa::block_attn_scratch_bytes(*d, DSA_MAX_BLOCK_QUERIES);
     default:
       return 0;
   }
@@ -253,11 +314,62 @@ dsa_status dsa_sparse_attn_decode(const dsa_dims* d, const uint16_t* q, const ui
                                            n_split, part));
 }
 
+dsa_status dsa_quantize_fp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* x8,
+                            float* scale, uint16_t* xhat, void* stream) {
+  if (rows < 0 || cols < 1 || cols > 128) return DSA_ERR_DIMS;
+  if (!x || !x8 || !scale || !xhat) return DSA_ERR_NULL;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(scale) || !aligned16(xhat)) return DSA_ERR_ALIGN;
+  dsa_status s = check_device();
+  if (s != DSA_OK) return s;
+  return from_cuda(dsa::launch_quantize_fp8(x, rows, cols, x8, scale, xhat,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_index_scores_fp8(const dsa_dims* d, const uint8_t* q8, const float* q_scale,
+                                const uint8_t* k8, const float* k_scale, const float* w_idx,
+                                float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  dsa_status s = check_dims(d, false, true);
+  if (s != DSA_OK) return s;
+  if (!q8 || !q_scale || !k8 || !k_scale || !w_idx || !scores) return DSA_ERR_NULL;
+  if (!aligned16(q8) || !aligned16(q_scale) || !aligned16(k8) || !aligned16(k_scale) ||
+      !aligned16(w_idx) || !aligned16(scores) || ld % 4 != 0)
+    return DSA_ERR_ALIGN;
+  if (ld < d->ctx_len) return DSA_ERR_DIMS;
+  if ((s = check_ws(*d, DSA_WS_INDEX_SCORES, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  return from_cuda(dsa::launch_index_scores_fp8(*d, q8, q_scale, k8, k_scale, w_idx, scores, ld,
+                                                static_cast<WsHeader*>(ws), st));
+}
+
+dsa_status dsa_sparse_attn_block(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
+                                 const uint16_t* rope, const int32_t* idx, uint16_t* out,
+                                 float* lse, int32_t block_queries, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  dsa_status s = check_dims(d, true, false);
+  if (s != DSA_OK) return s;
+  if (block_queries < 1 || block_queries > DSA_MAX_BLOCK_QUERIES) return DSA_ERR_DIMS;
+  if (!q || !latent || !rope || !idx || !out) return DSA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(idx) ||
+      !aligned16(out) || (lse && !aligned16(lse)))
+    return DSA_ERR_ALIGN;
+  if ((s = check_ws(*d, DSA_WS_BLOCK_ATTN, ws, ws_bytes)) != DSA_OK) return s;
+  if ((s = check_device()) != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  if (d->n_q == 0) return DSA_OK;
+  return from_cuda(dsa::launch_block_attn(*d, q, latent, rope, idx, out, lse, block_queries,
+                                          static_cast<WsHeader*>(ws),
+                                          static_cast<char*>(ws) + dsa::kWsHeaderBytes, st));
+}
+
 dsa_status dsa_decode_layer(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
                             const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                             const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                             void* ws, size_t ws_bytes, void* stream) {
-  dsa_status s = check_dims(d, true, true);
+  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
@@ -276,7 +388,7 @@ dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_
                              const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                              const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                              void* ws, size_t ws_bytes, void* stream) {
-  dsa_status s = check_dims(d, true, true);
+  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
@@ -295,7 +407,7 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const ui
                                   const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                                   const dsa_device_tensors* dev, void* ws, size_t ws_bytes,
                                   void* const streams[3], void* const events[2], int32_t n_sub) {
-  dsa_status s = check_dims(d, true, true);
+  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out || !dev || !streams || !events)
     return DSA_ERR_NULL;

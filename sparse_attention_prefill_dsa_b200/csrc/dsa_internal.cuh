@@ -73,6 +73,12 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
 cudaError_t launch_index_scores(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_idx,
                                 const float* w_idx, float* scores, int64_t ld, WsHeader* ws,
                                 cudaStream_t st);
+// FP8 indexer: e4m3 codes with per-row power-of-two scales (quantize first).
+cudaError_t launch_index_scores_fp8(const dsa_dims& d, const uint8_t* q8, const float* q_scale,
+                                    const uint8_t* k8, const float* k_scale, const float* w_idx,
+                                    float* scores, int64_t ld, WsHeader* ws, cudaStream_t st);
+cudaError_t launch_quantize_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* x8,
+                                float* scale, uint16_t* xhat, cudaStream_t st);
 cudaError_t launch_key_norm_max(const dsa_dims& d, const uint16_t* k_idx, WsHeader* ws,
                                 cudaStream_t st);
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld,
@@ -105,6 +111,15 @@ inline size_t attn_split_bytes(int n_q, int n_split, int H, int DC) {
 // DSA_OK when the current device is an sm_100 GPU, else DSA_ERR_DEVICE (or
 // DSA_ERR_CUDA when the runtime cannot say). Cached per device.
 dsa_status check_current_device();
+
+// Block-sparse attention over groups of qb (1 or 2) neighbouring queries:
+// the union of each group's selections (built into `scratch`, of
+// block_attn_scratch_bytes(d, qb) bytes, 16-byte aligned), then QK^T / PV on
+// the union with per-query masks.
+size_t block_attn_scratch_bytes(const dsa_dims& d, int qb);
+cudaError_t launch_block_attn(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
+                              const uint16_t* rope, const int32_t* idx, uint16_t* out, float* lse,
+                              int qb, WsHeader* ws, void* scratch, cudaStream_t st);
 
 // The bounded-wait self-test (one CTA, two warps on mbarriers nothing signals).
 cudaError_t launch_bounded_wait_selftest(WsHeader* ws, long long* cycles, cudaStream_t st);

@@ -36,6 +36,8 @@
 // workspace, all roles stop, outstanding TMA loads and MMAs are drained, and
 // TMEM is freed before the CTA exits.
 #include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -47,29 +49,34 @@ namespace {
 
 using namespace sm100;
 
-template <int HI, int DI>
+// FP8: the operands are e4m3 codes (1 byte, K = 32 per MMA, kind::f8f6f4)
+// with a power-of-two scale per key row and per (query, head) row; else bf16.
+template <int HI, int DI, bool FP8 = false>
 struct IdxCfg {
   static constexpr int kM = 128;                       // keys per tile (MMA M)
   static constexpr int kN = 256;                       // (query, head) columns (MMA N)
   static constexpr int kQB = kN / HI;                  // queries per block
-  static constexpr int kChunk = DI < 64 ? DI : 64;     // elements per swizzled row
+  static constexpr int kEB = FP8 ? 1 : 2;              // bytes per element
+  static constexpr int kChunk = DI * kEB < 128 ? DI : 128 / kEB;  // elements per swizzled row
   static constexpr int kNChunk = DI / kChunk;
-  static constexpr int kRowBytes = kChunk * 2;         // 128 or 64
-  static constexpr uint32_t kSwzCode = kRowBytes == 128 ? 2u : 4u;
+  static constexpr int kRowBytes = kChunk * kEB;       // 128, 64 or 32
+  static constexpr uint32_t kSwzCode = kRowBytes == 128 ? 2u : (kRowBytes == 64 ? 4u : 6u);
   static constexpr CUtensorMapSwizzle kSwzMap =
-      kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+      kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                       : (kRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
   static constexpr int kSbo = 8 * kRowBytes;           // bytes between 8-row groups
   static constexpr int kKChunkBytes = kM * kRowBytes;
   static constexpr int kQChunkBytes = kN * kRowBytes;
   static constexpr int kKTileBytes = kKChunkBytes * kNChunk;
   static constexpr int kQBytes = kQChunkBytes * kNChunk;
   static constexpr int kStages = 4;
-  static constexpr int kKSteps = DI / 16;
-  static constexpr int kStepsPerChunk = kChunk / 16;
+  static constexpr int kKPerMma = FP8 ? 32 : 16;       // elements of K per MMA (32 bytes)
+  static constexpr int kKSteps = DI / kKPerMma;
+  static constexpr int kStepsPerChunk = kChunk / kKPerMma;
   static constexpr int kTilesPerUnit = 32;             // key tiles per work unit (fewer for small chunks)
   static constexpr int kEpiWarps = 8;                  // warps 2-9
   static constexpr int kThreads = 32 * (2 + kEpiWarps);
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(kM, kN, false, false);
+  static constexpr uint32_t kIdesc = FP8 ? idesc_e4m3_f32(kM, kN) : idesc_bf16_f32(kM, kN, false, false);
   // shared memory carve (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
@@ -80,11 +87,14 @@ struct IdxCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffUnit = kOffMisc + 16;                     // int [kUnitRing]
   static constexpr int kSmemBytes = kOffUnit + 4 * kUnitRing + 1024;  // + alignment slack
-  static_assert(DI % 16 == 0 && kN % HI == 0 && HI <= 32 && 32 % HI == 0, "shape");
+  static_assert(DI % kKPerMma == 0 && kN % HI == 0 && HI <= 32 && 32 % HI == 0, "shape");
 };
 
 struct IdxParams {
   const float* w_idx;
+  const float* q_scale;  // FP8: [n_q * H_I] power-of-two scale of each (query, head) row
+  const float* k_scale;  // FP8: [ctx_len] scale of each key row
+  int ctx_len;
   float* scores;
   int64_t ld;
   int n_q, q_pos0;
@@ -131,11 +141,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kWaitLimitCycles) break;
 }
 
-template <int HI, int DI>
-__global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
+template <int HI, int DI, bool FP8>
+__global__ void __launch_bounds__(IdxCfg<HI, DI, FP8>::kThreads, 1)
     index_scores_tc(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_q, const IdxParams p) {
-  using C = IdxCfg<HI, DI>;
+  using C = IdxCfg<HI, DI, FP8>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -227,7 +237,10 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
       if (!ok) break;
       for (int e = lane; e < C::kN; e += 32) {
         const int i = qb * C::kQB + e / HI;
-        sW[wb * C::kN + e] = i < p.n_q ? __ldg(p.w_idx + static_cast<int64_t>(qb) * C::kN + e) : 0.f;
+        float wv = i < p.n_q ? __ldg(p.w_idx + static_cast<int64_t>(qb) * C::kN + e) : 0.f;
+        // FP8: w * s_q (a power of two: exact); the key's scale comes in the epilogue
+        if (FP8 && i < p.n_q) wv *= __ldg(p.q_scale + static_cast<int64_t>(qb) * C::kN + e);
+        sW[wb * C::kN + e] = wv;
       }
       mbar_arrive(&w_full[wb]);
       // the block's q_idx rows
@@ -294,7 +307,8 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
           const uint32_t off = (ks % C::kStepsPerChunk) * 32;
           const uint64_t a = dk + static_cast<uint64_t>((c * C::kKChunkBytes + off) >> 4);
           const uint64_t b = dq0 + static_cast<uint64_t>((c * C::kQChunkBytes + off) >> 4);
-          mma_bf16_ss_warp(d, a, b, C::kIdesc, ks > 0 ? 1u : 0u);
+          if constexpr (FP8) mma_f8_ss_warp(d, a, b, C::kIdesc, ks > 0 ? 1u : 0u);
+          else mma_bf16_ss_warp(d, a, b, C::kIdesc, ks > 0 ? 1u : 0u);
         }
         mma_commit_warp(&k_empty[st]);
         mma_commit_warp(&acc_full[buf]);
@@ -330,6 +344,9 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int s = kt * C::kM + key_local;
+        // FP8: the key row's scale, applied to the finished head sum (a power
+        // of two: relu(s_k x) = s_k relu(x), and the product is exact)
+        const float ks = FP8 ? (s < p.ctx_len ? __ldg(p.k_scale + s) : 0.f) : 1.f;
         // two 32-column groups per TMEM wait; the weights of a group are read
         // as float4 broadcasts
 #pragma unroll 1
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI>::kThreads, 1)
                 acc = fmaf(wv[qq * HI + j], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f), acc);
               const int i = qb * C::kQB + (col0 + qq * HI) / HI;
               if (i < p.n_q && s <= p.q_pos0 + i && DSA_IN_BOUNDS(p.ws, s, p.ld, 20))
-                p.scores[static_cast<int64_t>(i) * p.ld + s] = acc;
+                p.scores[static_cast<int64_t>(i) * p.ld + s] = FP8 ? acc * ks : acc;
             }
           }
         }
@@ -390,18 +407,29 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-template <int HI, int DI>
-cudaError_t launch(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_idx,
-                   const float* w_idx, float* scores, int64_t ld, WsHeader* ws, cudaStream_t st) {
-  using C = IdxCfg<HI, DI>;
+template <int HI, int DI, bool FP8>
+cudaError_t launch(const dsa_dims& d, const void* q_idx, const void* k_idx, const float* q_scale,
+                   const float* k_scale, const float* w_idx, float* scores, int64_t ld,
+                   WsHeader* ws, cudaStream_t st) {
+  using C = IdxCfg<HI, DI, FP8>;
   CUtensorMap tm_k, tm_q;
-  if (!make_tmap_bf16_2d(&tm_k, k_idx, DI, static_cast<uint64_t>(d.ctx_len), C::kChunk, C::kM,
+  if (FP8) {
+    if (!make_tmap_u8_2d(&tm_k, k_idx, DI, static_cast<uint64_t>(d.ctx_len), C::kChunk, C::kM,
                          C::kSwzMap) ||
-      !make_tmap_bf16_2d(&tm_q, q_idx, DI, static_cast<uint64_t>(d.n_q) * HI, C::kChunk, C::kN,
+        !make_tmap_u8_2d(&tm_q, q_idx, DI, static_cast<uint64_t>(d.n_q) * HI, C::kChunk, C::kN,
                          C::kSwzMap))
+      return cudaErrorInvalidValue;
+  } else if (!make_tmap_bf16_2d(&tm_k, k_idx, DI, static_cast<uint64_t>(d.ctx_len), C::kChunk,
+                                C::kM, C::kSwzMap) ||
+             !make_tmap_bf16_2d(&tm_q, q_idx, DI, static_cast<uint64_t>(d.n_q) * HI, C::kChunk,
+                                C::kN, C::kSwzMap)) {
     return cudaErrorInvalidValue;
+  }
   IdxParams p;
   p.w_idx = w_idx;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.ctx_len = d.ctx_len;
   p.scores = scores;
   p.ld = ld;
   p.n_q = d.n_q;
@@ -425,11 +453,55 @@ cudaError_t launch(const dsa_dims& d, const uint16_t* q_idx, const uint16_t* k_i
   // The CTA owns all 512 TMEM columns of its SM: ask for enough shared memory
   // that a second CTA can never be resident beside it.
   const int smem = C::kSmemBytes > kOneCtaPerSmSmem ? C::kSmemBytes : kOneCtaPerSmSmem;
-  cudaError_t e = cudaFuncSetAttribute(index_scores_tc<HI, DI>,
+  cudaError_t e = cudaFuncSetAttribute(index_scores_tc<HI, DI, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  index_scores_tc<HI, DI><<<grid, C::kThreads, smem, st>>>(tm_k, tm_q, p);
+  index_scores_tc<HI, DI, FP8><<<grid, C::kThreads, smem, st>>>(tm_k, tm_q, p);
   return cudaGetLastError();
+}
+
+// e4m3 codes of bf16 rows (one warp per row of `cols` <= 128 values): the
+// row's scale is the smallest power of two s with max|x| <= 448 s, the code
+// is x / s rounded to the nearest e4m3 value (ties to even, the hardware
+// conversion), and xhat = code * s as bf16 (exact).
+__global__ void quantize_fp8_kernel(const uint16_t* __restrict__ x, int64_t rows, int cols,
+                                    uint8_t* __restrict__ x8, float* __restrict__ scale,
+                                    uint16_t* __restrict__ xhat) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const uint16_t* xr = x + r * cols;
+  float v[4];
+  float amax = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = lane * 4 + u;
+    v[u] = c < cols ? bf16_to_f32(xr[c]) : 0.f;
+    amax = fmaxf(amax, fabsf(v[u]));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  // k: 448 * 2^k >= amax with k minimal; amax = m * 2^E, m in [1, 2):
+  // k = E - 8 when m <= 1.75, else E - 7 (448 = 1.75 * 2^8)
+  int k = 0;
+  if (amax > 0.f) {
+    int E;
+    const float m = frexpf(amax, &E) * 2.f;  // amax = m * 2^(E-1)
+    E -= 1;
+    k = m <= 1.75f ? E - 8 : E - 7;
+  }
+  if (lane == 0) scale[r] = ldexpf(1.f, k);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = lane * 4 + u;
+    if (c >= cols) break;
+    const float q = ldexpf(v[u], -k);  // exact
+    const __nv_fp8_storage_t code = __nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3);
+    x8[r * cols + c] = static_cast<uint8_t>(code);
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(code, __NV_E4M3);
+    const float deq = ldexpf(__half2float(__half(hr)), k);
+    xhat[r * cols + c] = static_cast<uint16_t>(__float_as_uint(deq) >> 16);
+  }
 }
 
 }  // namespace
@@ -438,10 +510,31 @@ cudaError_t launch_index_scores(const dsa_dims& d, const uint16_t* q_idx, const 
                                 const float* w_idx, float* scores, int64_t ld, WsHeader* ws,
                                 cudaStream_t st) {
   if (d.n_idx_heads == 32 && d.d_idx == 128)
-    return launch<32, 128>(d, q_idx, k_idx, w_idx, scores, ld, ws, st);
+    return launch<32, 128, false>(d, q_idx, k_idx, nullptr, nullptr, w_idx, scores, ld, ws, st);
   if (d.n_idx_heads == 2 && d.d_idx == 32)
-    return launch<2, 32>(d, q_idx, k_idx, w_idx, scores, ld, ws, st);
+    return launch<2, 32, false>(d, q_idx, k_idx, nullptr, nullptr, w_idx, scores, ld, ws, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_index_scores_fp8(const dsa_dims& d, const uint8_t* q8, const float* q_scale,
+                                    const uint8_t* k8, const float* k_scale, const float* w_idx,
+                                    float* scores, int64_t ld, WsHeader* ws, cudaStream_t st) {
+  if (d.n_idx_heads == 32 && d.d_idx == 128)
+    return launch<32, 128, true>(d, q8, k8, q_scale, k_scale, w_idx, scores, ld, ws, st);
+  if (d.n_idx_heads == 2 && d.d_idx == 32)
+    return launch<2, 32, true>(d, q8, k8, q_scale, k_scale, w_idx, scores, ld, ws, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quantize_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* x8,
+                                float* scale, uint16_t* xhat, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (cols < 1 || cols > 128) return cudaErrorInvalidValue;
+  const int threads = 256;
+  const int64_t blocks = (rows * 32 + threads - 1) / threads;
+  quantize_fp8_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(x, rows, cols, x8, scale,
+                                                                         xhat);
+  return cudaGetLastError();
 }
 
 }  // namespace dsa

@@ -25,19 +25,36 @@ void resolve() {
 
 }  // namespace
 
-bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
-                       uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+namespace {
+
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, uint32_t elem_bytes, const void* base,
+                  uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                  CUtensorMapSwizzle swizzle) {
   std::call_once(g_once, resolve);
   if (!g_encode) return false;
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint64_t strides[1] = {cols * elem_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
-                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+  const CUresult r = g_encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                       uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, cols, rows, box_cols,
+                      box_rows, swizzle);
+}
+
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                     uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, cols, rows, box_cols, box_rows,
+                      swizzle);
 }
 
 }  // namespace dsa

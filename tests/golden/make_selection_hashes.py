@@ -42,6 +42,10 @@ BLOCK_ROWS = 256
 # non-integral weights
 CASES = [(w.name, "ones" if w.kind == "ternary_ties" else "uniform") for w in workloads.WORKLOADS]
 CASES.append(("ties_4k_ctx8k", "uniform"))
+# the FP8 indexer variant's contract (the float64 scores of the dequantized
+# e4m3 rows) on the 2K- and 8K-query chunks and the tie stress
+CASES += [("chunk2k_ctx8k", "uniform", "fp8"), ("chunk8k_ctx17k", "uniform", "fp8"),
+          ("ties_4k_ctx8k", "ones", "fp8")]
 
 
 def inputs_digest(x: dict) -> str:
@@ -63,9 +67,14 @@ def selection_digests(idx: np.ndarray) -> tuple[str, list[str]]:
     return whole, blocks
 
 
-def oracle_selection(d, x, rows=None, threads=None, batch=None) -> np.ndarray:
+def oracle_selection(d, x, rows=None, threads=None, batch=None, fp8=False) -> np.ndarray:
     """The oracle's selection of the given rows (all rows by default), scored
-    and selected in batches of rows to bound the float64 score memory."""
+    and selected in batches of rows to bound the float64 score memory; with
+    fp8, under the FP8 indexer's contract (scores of the dequantized rows)."""
+    if fp8:
+        _, _, q_hat = oracle.quantize_fp8(x["q_idx"])
+        _, _, k_hat = oracle.quantize_fp8(x["k_idx"])
+        x = dict(x, q_idx=q_hat, k_idx=k_hat)
     if rows is None:
         rows = np.arange(d.n_q, dtype=np.int32)
     rows = np.asarray(rows, dtype=np.int32)
@@ -84,14 +93,14 @@ def oracle_source_digest() -> str:
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def case_key(name: str, w_mode: str) -> str:
-    return f"{name}:{w_mode}"
+def case_key(name: str, w_mode: str, variant: str = "") -> str:
+    return f"{name}:{w_mode}" + (f":{variant}" if variant else "")
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--only", action="append", default=[],
-                    help="NAME:MODE to (re)compute; default: every case")
+                    help="NAME:MODE[:VARIANT] to (re)compute; default: every case")
     ap.add_argument("--threads", type=int, default=0)
     args = ap.parse_args()
     oracle.build()
@@ -109,18 +118,20 @@ def main():
     data["oracle_source_sha256"] = oracle_source_digest()
     cases = data.setdefault("cases", {})
     todo = [c for c in CASES if not args.only or case_key(*c) in args.only]
-    for name, w_mode in todo:
+    for case in todo:
+        name, w_mode = case[0], case[1]
+        variant = case[2] if len(case) > 2 else ""
         wl = workloads.BY_NAME[name]
         d, x = workloads.workload_inputs(name, w_mode)
         t0 = time.time()
-        idx = oracle_selection(d, x, threads=args.threads or None)
+        idx = oracle_selection(d, x, threads=args.threads or None, fp8=variant == "fp8")
         whole, blocks = selection_digests(idx)
-        cases[case_key(name, w_mode)] = {
-            "workload": name, "w_mode": w_mode, "seed": wl.seed, "n_q": d.n_q,
+        cases[case_key(*case)] = {
+            "workload": name, "w_mode": w_mode, "variant": variant, "seed": wl.seed, "n_q": d.n_q,
             "ctx_len": d.ctx_len, "top_k": d.top_k, "inputs_sha256": inputs_digest(x),
             "selection_sha256": whole, "block_sha256": blocks,
         }
-        print(f"{name}:{w_mode}: {time.time() - t0:.0f} s", flush=True)
+        print(f"{case_key(*case)}: {time.time() - t0:.0f} s", flush=True)
         with open(OUT + ".tmp", "w") as f:
             json.dump(data, f, indent=1, sort_keys=True)
             f.write("\n")

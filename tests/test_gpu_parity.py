@@ -103,18 +103,23 @@ def test_layer_full_size_every_row(dsa, oracle_lib, case):
     element-wise on every row of the 256-, 2,048- and 4,096-query chunks and on
     512 rows spread over the 8,192- and 16,384-query chunks.
     """
+    import dataclasses
+
     g = _GOLDEN["cases"][case]
     name, w_mode = g["workload"], g["w_mode"]
+    fp8 = g.get("variant", "") == "fp8"
     d, x = workloads.workload_inputs(name, w_mode)
     assert _GOLDEN_MOD.inputs_digest(x) == g["inputs_sha256"], \
         "input recipe changed since the digests were written: rerun make_selection_hashes.py"
+    if fp8:  # the FP8 indexer's contract: the dequantized e4m3 rows
+        d = dataclasses.replace(d, flags=dsa.DSA_FLAG_FP8_INDEXER)
     out, lse, idx = run_layer(dsa, d, stage(x))
     whole, blocks = _GOLDEN_MOD.selection_digests(idx)
     if whole != g["selection_sha256"]:
         nb = _GOLDEN["block_rows"]
         bad = [b for b, (a, e) in enumerate(zip(blocks, g["block_sha256"])) if a != e]
         rows = np.arange(bad[0] * nb, min(d.n_q, (bad[0] + 1) * nb), dtype=np.int32)
-        ref = _GOLDEN_MOD.oracle_selection(d, x, rows=rows)
+        ref = _GOLDEN_MOD.oracle_selection(d, x, rows=rows, fp8=fp8)
         wrong = rows[~np.all(idx[rows] == ref, axis=1)]
         pytest.fail(f"{len(bad)} blocks of {nb} rows differ; first wrong rows {wrong[:8].tolist()}")
     if name in _ALL_ROWS:

@@ -349,12 +349,13 @@ def test_stored_selection_digests_match_the_oracle():
     nb = g["block_rows"]
     assert set(g["cases"]) == {mod.case_key(*c) for c in mod.CASES}
     for key, c in sorted(g["cases"].items()):
+        fp8 = c.get("variant", "") == "fp8"
         d, x = workloads.workload_inputs(c["workload"], c["w_mode"])
         assert mod.inputs_digest(x) == c["inputs_sha256"], key
         n_blocks = (d.n_q + nb - 1) // nb
         assert len(c["block_sha256"]) == n_blocks
         if d.n_q <= nb:
-            whole, _ = mod.selection_digests(mod.oracle_selection(d, x))
+            whole, _ = mod.selection_digests(mod.oracle_selection(d, x, fp8=fp8))
             assert whole == c["selection_sha256"], key
             continue
         # first block always; the last one too where the oracle is quick
@@ -363,7 +364,7 @@ def test_stored_selection_digests_match_the_oracle():
             rows = np.arange(b * nb, min(d.n_q, (b + 1) * nb), dtype=np.int32)
             if d.ctx_len > 20000:
                 rows = rows[:nb]
-            sel = mod.oracle_selection(d, x, rows=rows)
+            sel = mod.oracle_selection(d, x, rows=rows, fp8=fp8)
             _, digests = mod.selection_digests(sel)
             assert digests[0] == c["block_sha256"][b], (key, b)
 

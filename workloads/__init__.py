@@ -37,6 +37,7 @@ class Dims:
     d_idx: int
     top_k: int
     softmax_scale: float
+    flags: int = 0  # dsa_dims.flags of the C ABI (the oracle ignores it)
 
     @property
     def d_qk(self) -> int:
