@@ -258,6 +258,9 @@ def attn_variants(dsa, d, xd, idx, out, lse, flush, stream, steps):
         "per_query": lambda: dsa.dsa_sparse_attn_prefill(
             d, xd["q"], xd["latent"], xd["rope"], idx, out, lse, ws_for(dsa.DSA_WS_ATTN),
             stream=stream),
+        "sm_pair": lambda: dsa.dsa_sparse_attn_prefill(
+            dataclasses.replace(d, flags=dsa.DSA_FLAG_ATTN_PAIR), xd["q"], xd["latent"],
+            xd["rope"], idx, out, lse, ws_for(dsa.DSA_WS_ATTN), stream=stream),
         "decode_split": lambda: dsa.dsa_sparse_attn_decode(
             d, xd["q"], xd["latent"], xd["rope"], idx, out, lse, ws_for(dsa.DSA_WS_DECODE_ATTN),
             stream=stream),

@@ -64,8 +64,16 @@ typedef struct dsa_dims {
  * indexer: q_idx and k_idx are taken to their e4m3 form (dsa_quantize_fp8,
  * in the workspace), scored by dsa_index_scores_fp8, and the exact top-k
  * orders keys by the float64 contract of dsa_topk_select on the dequantized
- * rows. Every other call requires flags == 0. */
+ * rows. Calls other than those named here require flags == 0. */
 #define DSA_FLAG_FP8_INDEXER 1u
+/* dims.flags: dsa_sparse_attn_prefill and the prefill-layer calls run the
+ * attention on SM pairs (a thread-block cluster of two CTAs per query, each
+ * gathering half of every selected key's dims, so that two tiles fit in
+ * flight; the halves of S and P cross between the pair through distributed
+ * shared memory). Shapes without that kernel (the 4-head shape) and the
+ * decode calls ignore it. Outputs agree with the one-SM kernel within
+ * rounding; selections are unaffected. */
+#define DSA_FLAG_ATTN_PAIR 2u
 
 /* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):
  *   (n_heads, d_latent, d_rope)  in {(4, 64, 16), (32, 512, 64)}

@@ -140,6 +140,16 @@ dsa_status clear_header(void* ws, cudaStream_t st) {
   return from_cuda(cudaMemsetAsync(ws, 0, dsa::kWsHeaderBytes, st));
 }
 
+// The prefill attention: on SM pairs when the caller asks for it
+// (DSA_FLAG_ATTN_PAIR) and the shape has that kernel, else one SM per query.
+cudaError_t attention(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
+                      const uint16_t* rope, const int32_t* idx, uint16_t* out, float* lse,
+                      bool prefix_valid, WsHeader* h, cudaStream_t st) {
+  if ((d.flags & DSA_FLAG_ATTN_PAIR) != 0u && dsa::attn_pair_supported(d))
+    return dsa::launch_sparse_attn_pair(d, q, latent, rope, idx, out, lse, prefix_valid, h, st);
+  return dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, prefix_valid, h, st);
+}
+
 // The layer's kernels on validated arguments (the workspace header cleared
 // by the caller): scores -> exact top-k -> attention. The two key-norm passes
 // (max ||k_idx[s]|| for the top-k band, max ||[latent_s, rope_s]|| for the
@@ -193,7 +203,7 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
     return from_cuda(
         dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, true, h, st, n_split, part));
   }
-  return from_cuda(dsa::launch_sparse_attn(d, q, latent, rope, idx, out, lse, true, h, st));
+  return from_cuda(attention(d, q, latent, rope, idx, out, lse, true, h, st));
 }
 
 cudaError_t h2d(void* dst, const void* src, size_t bytes, cudaStream_t st) {
@@ -274,7 +284,7 @@ dsa_status dsa_topk_select(const dsa_dims* d, const float* scores, int64_t ld,
 dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
                                    const uint16_t* rope, const int32_t* idx, uint16_t* out,
                                    float* lse, void* ws, size_t ws_bytes, void* stream) {
-  dsa_status s = check_dims(d, true, false);
+  dsa_status s = check_dims(d, true, false, DSA_FLAG_ATTN_PAIR);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !idx || !out) return DSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(idx) ||
@@ -288,7 +298,7 @@ dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const u
   WsHeader* h = static_cast<WsHeader*>(ws);
   cudaError_t e = dsa::launch_attn_key_norm_max(*d, latent, rope, h, st);
   if (e != cudaSuccess) return DSA_ERR_CUDA;
-  return from_cuda(dsa::launch_sparse_attn(*d, q, latent, rope, idx, out, lse, false, h, st));
+  return from_cuda(attention(*d, q, latent, rope, idx, out, lse, false, h, st));
 }
 
 dsa_status dsa_sparse_attn_decode(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,
@@ -369,7 +379,7 @@ dsa_status dsa_decode_layer(const dsa_dims* d, const uint16_t* q, const uint16_t
                             const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                             const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                             void* ws, size_t ws_bytes, void* stream) {
-  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER);
+  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
@@ -388,7 +398,7 @@ dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_
                              const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                              const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                              void* ws, size_t ws_bytes, void* stream) {
-  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER);
+  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
@@ -407,7 +417,7 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const ui
                                   const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                                   const dsa_device_tensors* dev, void* ws, size_t ws_bytes,
                                   void* const streams[3], void* const events[2], int32_t n_sub) {
-  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER);
+  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out || !dev || !streams || !events)
     return DSA_ERR_NULL;

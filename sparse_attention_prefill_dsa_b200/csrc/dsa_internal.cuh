@@ -98,6 +98,12 @@ cudaError_t launch_sparse_attn(const dsa_dims& d, const uint16_t* q, const uint1
                                const uint16_t* rope, const int32_t* idx, uint16_t* out,
                                float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st,
                                int n_split = 1, void* part = nullptr);
+// The same attention on SM pairs (a cluster of two CTAs per query, each with
+// half of every key's dims), for the 32-head 512 + 64 shape only.
+bool attn_pair_supported(const dsa_dims& d);
+cudaError_t launch_sparse_attn_pair(const dsa_dims& d, const uint16_t* q, const uint16_t* latent,
+                                    const uint16_t* rope, const int32_t* idx, uint16_t* out,
+                                    float* lse, bool prefix_valid, WsHeader* ws, cudaStream_t st);
 // The split the decode entry points use: as many ranges per query as leave no
 // SM idle, at most one per 128-key tile of top_k.
 int attn_decode_split(const dsa_dims& d);

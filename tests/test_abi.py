@@ -105,7 +105,7 @@ def test_host_validation_before_any_device_call(dsa):
     bad.n_q = d.n_q + 1
     assert _layer(dsa, bad) == dsa.DSA_ERR_CAUSAL
     for field, val in (("top_k", 0), ("top_k", 2049), ("ctx_len", 49153), ("n_heads", 8),
-                       ("d_latent", 256), ("n_idx_heads", 64), ("flags", 2), ("n_q", -1),
+                       ("d_latent", 256), ("n_idx_heads", 64), ("flags", 4), ("n_q", -1),
                        ("softmax_scale", 0.0)):
         bad = dsa.make_dims(d)
         setattr(bad, field, val)
