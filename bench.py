@@ -300,8 +300,6 @@ def run_ours(args):
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     x = workloads.generate(d, rank_seed(wl.seed, rank), wl.kind, w_mode)
     if args.fp8_indexer:  # the FP8 indexer variant of the layer (its own selection contract)
-        import dataclasses
-
         d = dataclasses.replace(d, flags=dsa.DSA_FLAG_FP8_INDEXER)
     stream = torch.cuda.current_stream()
 

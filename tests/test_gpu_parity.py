@@ -423,7 +423,7 @@ def test_argument_errors_launch_nothing(dsa):
     assert dsa.dsa_prefill_layer(d, *bad) == dsa.DSA_ERR_ALIGN
     assert dsa.dsa_prefill_layer(d, *args, workspace_bytes=nbytes - 1) == dsa.DSA_ERR_WORKSPACE
     for field, val, code in (("top_k", 4096, dsa.DSA_ERR_DIMS), ("n_heads", 16, dsa.DSA_ERR_DIMS),
-                             ("d_idx", 64, dsa.DSA_ERR_DIMS), ("flags", 1, dsa.DSA_ERR_DIMS),
+                             ("d_idx", 64, dsa.DSA_ERR_DIMS), ("flags", 4, dsa.DSA_ERR_DIMS),
                              ("n_q", d.n_q + 1, dsa.DSA_ERR_CAUSAL)):
         dd = dsa.make_dims(d)
         setattr(dd, field, val)
