@@ -46,7 +46,15 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel inside the layer on a workload, from one ncu capture of that launch
 # (bench.py --layer-only on the same workload). An entry is removed whenever
 # its kernel changes after the capture.
-PROFILED_DRAM_BYTES_PER_LAUNCH: dict = {}
+# key: (CUDA kernel, workload); value: bytes per launch
+PROFILED_DRAM_BYTES_PER_LAUNCH: dict = {
+    ("index_scores_tc", "chunk8k_ctx17k"): 256_241_408 + 394_494_464,
+    ("topk_kernel", "chunk8k_ctx17k"): 514_805_760 + 57_556_736,
+    ("sparse_attn_tc", "chunk8k_ctx17k"): 389_857_536 + 242_595_840,
+}
+# the CUDA kernel behind each timed entry point (the layer's own launch configuration)
+KERNEL_OF = {"index_scores": "index_scores_tc", "topk_select": "topk_kernel",
+             "sparse_attn": "sparse_attn_tc"}
 
 KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
 # (the FP8 indexer variant adds the e4m3 forms of the keys and of the queries)
@@ -454,8 +462,11 @@ def run_ours(args):
     # the current kernel on this workload exists
     dom_name = max(per_kernel, key=per_kernel.get)
     r = rates[dom_name]
-    prof = PROFILED_DRAM_BYTES_PER_LAUNCH.get((dom_name, wl.name))
-    roof = {"kernel": dom_name, "bound": r["bound"], "achieved": r["achieved"],
+    kernel = KERNEL_OF[dom_name]
+    if dom_name == "sparse_attn" and d.flags & dsa.DSA_FLAG_ATTN_PAIR:
+        kernel = "sparse_attn_pair"
+    prof = PROFILED_DRAM_BYTES_PER_LAUNCH.get((kernel, wl.name)) if not args.fp8_indexer else None
+    roof = {"kernel": kernel, "bound": r["bound"], "achieved": r["achieved"],
             "peak": peaks["bf16_tflops"] if r["bound"] == "tensor" else peaks["hbm_gbs"],
             "unit": r["unit"], "frac": r["frac"],
             "traffic": prof if prof else None,
