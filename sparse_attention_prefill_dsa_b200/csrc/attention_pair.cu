@@ -306,13 +306,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[B::kSFull + b], 1);
       mbar_init(&bars[B::kSEmpty + b], C::kSoftmaxThreads);
-      mbar_init(&bars[B::kRecvFull + b], C::kSoftmaxThreads);        // the other CTA's threads
-      mbar_init(&bars[B::kPFull + b], 2 * C::kSoftmaxThreads);       // both CTAs' threads
-      mbar_init(&bars[B::kOReady + b], C::kSoftmaxThreads);
+      // one arrival per softmax warp: the other CTA's warps, or both CTAs' warps
+      mbar_init(&bars[B::kRecvFull + b], C::kSoftmaxWarps);
+      mbar_init(&bars[B::kPFull + b], 2 * C::kSoftmaxWarps);
+      mbar_init(&bars[B::kOReady + b], C::kSoftmaxWarps);
       mbar_init(&bars[B::kOFull + b], 1);
       mbar_init(&bars[B::kOEmpty + b], C::kSoftmaxThreads);
       mbar_init(&bars[B::kExch + b], C::kSoftmaxThreads);
-      mbar_init(&bars[B::kLFull + b], 2 * C::kSoftmaxThreads);
+      mbar_init(&bars[B::kLFull + b], 2 * C::kSoftmaxWarps);
     }
     mbar_init(&bars[B::kOStep], 1);
     mbar_init(&bars[B::kMmaDone], 1);
@@ -431,14 +432,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
           mma_bf16_ss_warp(d_s, pdesc_add(drope, sl * C::kRopeBytes + ks * 32), pdesc_add(dqr, ks * 32),
                            C::kIdescQK, ks > 0 ? 1u : 0u);
         mma_commit_warp(&bars[B::kRopeEmpty + sl]);
-        if (!(ok = pair_qk(p, abort_flag, bars, dpair_k, dq, tc, 0, d_s))) break;
+        // all of QK^T(t) first, so that the softmax of tile t runs while the
+        // tensor pipe does PV(t-1); two tiles in flight keep the gather ahead
+        for (int mb = 0; mb < C::MB && ok; ++mb) ok = pair_qk(p, abort_flag, bars, dpair_k, dq, tc, mb, d_s);
+        if (!ok) break;
+        mma_commit_warp(&bars[B::kSFull + sb]);
         if (pend && !(ok = pair_pv(p, abort_flag, bars, tmem_base, dpair_mn, dp, pend_tc, pend_qi, pend_first,
                                    pend_last)))
           break;
         pend = false;
-        for (int mb = 1; mb < C::MB && ok; ++mb) ok = pair_qk(p, abort_flag, bars, dpair_k, dq, tc, mb, d_s);
-        if (!ok) break;
-        mma_commit_warp(&bars[B::kSFull + sb]);
         pend = true;
         pend_tc = tc;
         pend_qi = qi;
@@ -532,7 +534,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
                         __float_as_uint(xp[3]));
           st_cluster_v4(dst + 16, __float_as_uint(xp[4]), __float_as_uint(xp[5]), __float_as_uint(xp[6]),
                         __float_as_uint(xp[7]));
-          mbar_arrive_remote(rRecvFull + sb * 8);
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(rRecvFull + sb * 8);  // releases the warp's stores
         }
         ok = pwarp_wait_cluster(&bars[B::kRecvFull + sb], (tc >> 1) & 1, abort_flag, p.ws, 71);
         if (!ok) break;
@@ -612,8 +615,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
         }
         fence_proxy_async_all();
         tc_fence_before();
-        mbar_arrive(&bars[B::kPFull + pb]);
-        mbar_arrive_remote(rPFull + pb * 8);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars[B::kPFull + pb]);
+          mbar_arrive_remote(rPFull + pb * 8);
+        }
         ok = pwarp_wait_cluster(&bars[B::kPFull + pb], (tc >> 1) & 1, abort_flag, p.ws, 73);
         if (!ok) break;
         // rescale O^T columns of every head whose maximum grew (this CTA's or
@@ -643,7 +649,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
           }
         }
         tc_fence_before();
-        mbar_arrive(&bars[B::kOReady + pb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B::kOReady + pb]);
       }
       if (!ok) break;
       // ---- epilogue of query i
@@ -668,8 +675,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::kThreads, 1
           p.lse[static_cast<int64_t>(i) * H + 16 * rank + lane] =
               l > 0.f ? (m_lane + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
-      mbar_arrive(&bars[B::kLFull + ob]);
-      mbar_arrive_remote(rLFull + ob * 8);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars[B::kLFull + ob]);
+        mbar_arrive_remote(rLFull + ob * 8);
+      }
       ok = pwarp_wait_cluster(&bars[B::kLFull + ob], (qi >> 1) & 1, abort_flag, p.ws, 77);
       if (!ok) break;
 #pragma unroll 1

@@ -86,8 +86,6 @@ struct Scratch {
   double wd[kWarps];
   int bc[4];
   float bf[4];
-  int alpha[kWarps];         // per warp: max over its heads of E1(q_j) - lsb_min(q_j)
-  unsigned int badbits[32];  // band keys the tensor-core re-score could not certify exact
 };
 
 __device__ __forceinline__ float canon(float f) { return f == 0.f ? 0.f : f; }  // -0 -> +0
@@ -366,31 +364,6 @@ __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int
   }
 }
 
-// Exponent of the last mantissa bit of a nonzero bf16 value (its ulp is
-// 2^result): e - 7 for a normal value with exponent e, -133 for a subnormal;
-// +1000 for zero, so that a minimum over values skips zeros.
-__device__ __forceinline__ int bf16_lsb_exp(uint16_t b) {
-  const int field = (b >> 7) & 0xFF;
-  if ((b & 0x7FFFu) == 0u) return 1000;
-  return field == 0 ? -133 : field - 127 - 7;
-}
-
-// Exponent e with |x| < 2^(e+1) for a nonzero bf16 value (-1000 for zero).
-__device__ __forceinline__ int bf16_top_exp(uint16_t b) {
-  const int field = (b >> 7) & 0xFF;
-  if ((b & 0x7FFFu) == 0u) return -1000;
-  return field == 0 ? -127 : field - 127;
-}
-
-// D (8 x 8) += A (8 x 4, row-major) * B (4 x 8, column-major) in float64 on
-// the tensor cores; lane l holds A[l/4][l%4], B[l%4][l/4] and
-// D[l/4][2(l%4)], D[l/4][2(l%4)+1].
-__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-               : "+d"(d[0]), "+d"(d[1])
-               : "d"(a), "d"(b));
-}
-
 // Row data of a key for the float64 re-score: lane l holds dims 4l..4l+3.
 __device__ __forceinline__ uint2 load_key_part(const uint16_t* __restrict__ k_idx, int key, int DI) {
   const int lane = threadIdx.x & 31;
@@ -464,88 +437,6 @@ __device__ __forceinline__ double rescore4(const uint32_t* __restrict__ qhi, dou
         sum = __dadd_rn(sum, v.y);  // HI is even
       }
     }
-  }
-  __syncwarp();
-  return sum;
-}
-
-// Contract scores of eight keys (one warp) with the head dots on the float64
-// tensor cores. A head dot of the contract is a sequential float64 chain of
-// exact products (bf16 x bf16); every partial sum of it is an integer
-// multiple of U = 2^(lsb_min(q_j) + lsb_min(k)) no larger in magnitude than
-// sum |q k| < 2^(E1(q_j) + E(max |k|) + 1). When that bound is below 2^53 U,
-// every partial sum in any order is a float64 value, nothing rounds, and the
-// chain equals the exact dot, which the tensor cores then return exactly:
-// alpha_max (the row's largest E1(q_j) - lsb_min(q_j)) + beta (the key's
-// E(max|k|) + 1 - lsb_min(k)) <= 53. Lane e < 8 returns key e's score and
-// sets *exact; other lanes return 0. raw[e] is key e's row part
-// (load_key_part); kst holds 8 x 128 words (the keys' float64 high words,
-// 16-byte groups XOR-swizzled by key so that the B loads hit 32 banks), and
-// afterwards the [8][34] products of the head sum.
-template <int DI>
-__device__ __forceinline__ double rescore8_tc(const uint32_t* __restrict__ qhi, int qstride,
-                                             float w_pre, const uint2 (&raw)[8],
-                                             uint32_t* __restrict__ kst, int HI, int alpha_max,
-                                             bool* exact) {
-  const int lane = threadIdx.x & 31;
-  int beta_mine = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    int top = -1000, low = 1000;
-    if (lane * 4 < DI) {
-      const uint32_t w[2] = {raw[e].x, raw[e].y};
-      uint32_t h[4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const uint16_t b0 = static_cast<uint16_t>(w[u] & 0xFFFFu), b1 = static_cast<uint16_t>(w[u] >> 16);
-        h[2 * u] = static_cast<uint32_t>(__double2hiint(bf16_to_f64(b0)));
-        h[2 * u + 1] = static_cast<uint32_t>(__double2hiint(bf16_to_f64(b1)));
-        top = max(top, max(bf16_top_exp(b0), bf16_top_exp(b1)));
-        low = min(low, min(bf16_lsb_exp(b0), bf16_lsb_exp(b1)));
-      }
-      *reinterpret_cast<uint4*>(kst + e * 128 + ((lane * 4) ^ (e * 4))) = make_uint4(h[0], h[1], h[2], h[3]);
-    }
-    top = __reduce_max_sync(0xffffffffu, top);
-    low = __reduce_min_sync(0xffffffffu, low);
-    const int beta = (top > -1000 && low < 1000) ? top + 1 - low : 0;  // an all-zero key is exact
-    if (lane == e) beta_mine = beta;
-  }
-  __syncwarp();
-  double acc[4][2];
-#pragma unroll
-  for (int m = 0; m < 4; ++m) acc[m][0] = acc[m][1] = 0.0;
-  const int g = lane >> 2, c = lane & 3;
-  const uint32_t* kb = kst + g * 128;
-  const int kx = (g * 4) & 31;
-#pragma unroll 4
-  for (int k0 = 0; k0 < DI; k0 += 4) {
-    const double b = __hiloint2double(static_cast<int>(kb[((k0 ^ kx)) + c]), 0);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      if (8 * m < HI) {
-        const double av = __hiloint2double(static_cast<int>(qhi[(8 * m + g) * qstride + k0 + c]), 0);
-        dmma_8x8x4(acc[m], av, b);
-      }
-    }
-  }
-  __syncwarp();
-  // p = w_j * relu(d) for head j = 8m + g and keys 2c, 2c + 1, into [key][34]
-  double* prod = reinterpret_cast<double*>(kst);
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int j = 8 * m + g;
-    const double wj = static_cast<double>(__shfl_sync(0xffffffffu, w_pre, j & 31));
-    if (j < HI) {
-#pragma unroll
-      for (int i = 0; i < 2; ++i) prod[(2 * c + i) * 34 + j] = __dmul_rn(wj, acc[m][i] > 0.0 ? acc[m][i] : 0.0);
-    }
-  }
-  __syncwarp();
-  double sum = 0.0;
-  if (lane < 8) {
-    const double* pe = prod + lane * 34;
-    for (int j = 0; j < HI; ++j) sum = __dadd_rn(sum, pe[j]);
-    *exact = alpha_max + beta_mine <= 53;
   }
   __syncwarp();
   return sum;
@@ -627,12 +518,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       }
     }
     double acc = 0.0;
-    int alpha_w = -1000;
 #pragma unroll
     for (int u = 0; u < kHeadsPerWarp; ++u) {
       const int j = w0 + u * kWarps;
-      double ss = 0.0, s1 = 0.0;
-      int lmin = 1000;
+      double ss = 0.0;
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         const int pr = l0 + 32 * t;
@@ -644,29 +533,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
           qhi[j * qstride + 2 * pr + 1] = static_cast<uint32_t>(__double2hiint(hi));
           ss += lo * lo;
           ss += hi * hi;
-          s1 += fabs(lo) + fabs(hi);
-          lmin = min(lmin, min(bf16_lsb_exp(static_cast<uint16_t>(v & 0xFFFFu)),
-                               bf16_lsb_exp(static_cast<uint16_t>(v >> 16))));
         }
       }
 #pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      }
-      lmin = __reduce_min_sync(0xffffffffu, lmin);
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float wj = __shfl_sync(0xffffffffu, w_pre, j & 31);
-      if (j < a.HI) {
-        acc += fabs(static_cast<double>(wj)) * sqrt(ss);
-        // ||q_j||_1 < 2^E1 (two bits of slack over its float64 exponent)
-        const int e1 = s1 > 0.0 ? ((__double2hiint(s1) >> 20) & 0x7FF) - 1023 + 2 : -1000;
-        if (s1 > 0.0) alpha_w = max(alpha_w, e1 - lmin);
-      }
+      if (j < a.HI) acc += fabs(static_cast<double>(wj)) * sqrt(ss);
     }
-    if (l0 == 0) {
-      sm.wd[w0] = acc;
-      sm.alpha[w0] = alpha_w;
-    }
+    if (l0 == 0) sm.wd[w0] = acc;
   }
   for (int s = n4 + threadIdx.x; s < n; s += kThreads) sc[s] = __ldg(srow + s);
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -773,63 +647,24 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     // re-score the collected band four keys per warp call (the next four rows
     // are loaded while the current ones are scored), rank it by (X desc,
     // index asc), and mark the row: kept band keys -> +inf, dropped -> -inf
-    // pass 1: eight keys per warp call with the head dots on the float64
-    // tensor cores (4 KB of key staging per warp), each result certified
-    // exact (rescore8_tc) or flagged in badbits
-    int alpha_max = -1000;
-    for (int w = 0; w < kWarps; ++w) alpha_max = max(alpha_max, sm.alpha[w]);
-    const int tcw = (kBins * 4 + kCandCap * 4 + a.kst_extra) / 4096;  // warps with 4 KB of staging
-    if (threadIdx.x < 32) sm.badbits[threadIdx.x] = 0u;
-    __syncthreads();
-    {
-      uint32_t* kst8 = kst_all + warp * 1024;
-      for (int b = warp < tcw ? 8 * warp : tot_band; b < tot_band; b += 8 * tcw) {
-        uint2 raw[8];
+    int b = warp < kw ? 4 * warp : tot_band;
+    uint2 raw[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) raw[e] = load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)], DI);
-        bool exact = false;
-        const double xl = DI == 128 ? rescore8_tc<128>(qhi, qstride, w_pre, raw, kst8, HI, alpha_max, &exact)
-                                    : rescore8_tc<32>(qhi, qstride, w_pre, raw, kst8, HI, alpha_max, &exact);
-        if (lane < 8 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, a.bcap, 4)) {
-          if (exact) bx[b + lane] = d2key(xl);
-          else atomicOr(&sm.badbits[(b + lane) >> 5], 1u << ((b + lane) & 31));
-        }
-      }
-    }
-    __syncthreads();
-    // pass 2 (keys pass 1 could not certify, rare): the sequential float64
-    // chains, four keys per warp call; the r-th such key goes to warp
-    // (r / 4) % kw
-    {
-      int r = 0, grp = 0;
-      int keys4[4];
-      const int nwords = (tot_band + 31) >> 5;
-      for (int wd = 0; wd < nwords; ++wd) {
-        unsigned int bits = sm.badbits[wd];
-        while (bits) {
-          const int pos = wd * 32 + __ffs(bits) - 1;
-          bits &= bits - 1;
-          if (((r >> 2) % kw) == warp) keys4[grp++] = pos;
-          ++r;
-          if (grp == 4) {
-            uint2 raw[4];
+    for (int e = 0; e < 4; ++e)
+      raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)], DI) : make_uint2(0u, 0u);
+    for (; b < tot_band; b += 4 * kw) {
+      const int bn = b + 4 * kw;
+      uint2 nraw[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) raw[e] = load_key_part(a.k_idx, bidx[keys4[e]], DI);
-            const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
-                                        : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
-            if (lane < 4) bx[keys4[lane & 3]] = d2key(xl);
-            grp = 0;
-          }
-        }
-      }
-      if (warp < kw && grp > 0) {
-        uint2 raw[4];
+      for (int e = 0; e < 4; ++e)
+        nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)], DI)
+                                : make_uint2(0u, 0u);
+      const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
+                                  : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
+      if (lane < 4 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, a.bcap, 4))
+        bx[b + lane] = d2key(xl);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) raw[e] = load_key_part(a.k_idx, bidx[keys4[min(e, grp - 1)]], DI);
-        const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
-                                    : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
-        if (lane < grp) bx[keys4[lane & 3]] = d2key(xl);
-      }
+      for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
     }
     __syncthreads();
     // rank of each band key by (X desc, index asc): a warp takes four keys at
