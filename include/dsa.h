@@ -78,9 +78,9 @@ typedef struct dsa_dims {
 /* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):
  *   (n_heads, d_latent, d_rope)  in {(4, 64, 16), (32, 512, 64)}
  *   (n_idx_heads, d_idx)         in {(2, 32), (32, 128)}
- *   1 <= top_k <= 2048, ctx_len <= 49152                                       */
+ *   1 <= top_k <= 2048, ctx_len <= 131072                                      */
 #define DSA_MAX_TOPK 2048
-#define DSA_MAX_CTX 49152
+#define DSA_MAX_CTX 131072
 
 typedef int32_t dsa_status;
 #define DSA_OK 0
@@ -109,8 +109,12 @@ typedef int32_t dsa_status;
  * arguments). The first 256 bytes of every workspace hold the device status
  * word and per-call scalars; dsa_prefill_layer adds the float32 score matrix
  * [n_q, round_up(ctx_len, 128)] and an int32 selection [n_q, top_k] after
- * them. Workspace contents need no initialisation and are not preserved
- * between calls. */
+ * them. When the chunk's last query sees more than 49,152 keys
+ * (q_pos0 + n_q > 49152) the top-k selects in two passes -- the top_k of
+ * each of n_seg = ceil((q_pos0 + n_q) / 32768) key segments, then the top_k
+ * of those candidates -- and dsa_topk_select and the layer calls add an
+ * int32 candidate buffer [n_q, n_seg, top_k]. Workspace contents need no
+ * initialisation and are not preserved between calls. */
 size_t dsa_workspace_size(const dsa_dims* dims, int32_t which);
 
 /* Lightning-indexer scores (component-table row "DSA indexer" of the feedman.me

@@ -50,7 +50,7 @@ DSA_FLAG_ATTN_PAIR = 2
 DSA_MAX_BLOCK_QUERIES = 2
 
 DSA_MAX_TOPK = 2048
-DSA_MAX_CTX = 49152
+DSA_MAX_CTX = 131072
 
 EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_sparse_attn_prefill", "dsa_prefill_layer", "dsa_device_status",

@@ -93,9 +93,10 @@ size_t decode_part_bytes(const dsa_dims& d) {
 // indexer the keys' e4m3 form (it depends on the cache only, so sub-chunks of
 // one chunk find it at the same place); the float32 scores; the selection;
 // with the FP8 indexer the queries' e4m3 form; for decode the split
-// attention's partials. Without either option this is header | scores | idx.
+// attention's partials; for rows of more than 49,152 keys the top-k's
+// candidate buffer. Without these this is header | scores | idx.
 struct LayerWs {
-  size_t kfp8, scores, idx, qfp8, part, total;
+  size_t kfp8, scores, idx, qfp8, part, cand, total;
 };
 
 LayerWs layer_ws(const dsa_dims& d, bool decode) {
@@ -107,7 +108,8 @@ LayerWs layer_ws(const dsa_dims& d, bool decode) {
   w.idx = w.scores + layer_scores_bytes(d);
   w.qfp8 = w.idx + (f8 || decode ? r256(idx_bytes) : idx_bytes);
   w.part = w.qfp8 + (f8 ? fp8_rows_bytes(static_cast<size_t>(d.n_q) * d.n_idx_heads, d.d_idx) : 0);
-  w.total = w.part + (decode ? decode_part_bytes(d) : 0);
+  w.cand = w.part + (decode ? decode_part_bytes(d) : 0);
+  w.total = w.cand + dsa::topk_cand_bytes(d);
   return w;
 }
 
@@ -168,6 +170,7 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
   // The selection goes to the caller's idx_out when given, else to the
   // workspace region after the score matrix.
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.idx);
+  void* cand = static_cast<char*>(ws) + w.cand;
   cudaError_t e = cudaSuccess;
   if (fp8_indexer(d)) {
     // FP8 indexer: the e4m3 forms of k_idx (once per cache) and q_idx; the
@@ -186,7 +189,7 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
     if (e == cudaSuccess)
       e = dsa::launch_index_scores_fp8(d, q8.x8, q8.scale, k8.x8, k8.scale, w_idx, scores, ld, h, st);
     if (e != cudaSuccess) return DSA_ERR_CUDA;
-    e = dsa::launch_topk(d, scores, ld, q8.xhat, k8.xhat, w_idx, idx, h, st);
+    e = dsa::launch_topk(d, scores, ld, q8.xhat, k8.xhat, w_idx, idx, h, cand, st);
   } else {
     if (!norms_ready) {
       e = dsa::launch_key_norm_max(d, k_idx, h, st);
@@ -194,7 +197,7 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
     }
     if (e == cudaSuccess) e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
     if (e != cudaSuccess) return DSA_ERR_CUDA;
-    e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, st);
+    e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, cand, st);
   }
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (decode) {
@@ -222,9 +225,10 @@ size_t dsa_workspace_size(const dsa_dims* d, int32_t which) {
   if (!d || d->n_q < 0 || d->ctx_len < 1) return 0;
   switch (which) {
     case DSA_WS_INDEX_SCORES:
-    case DSA_WS_TOPK:
     case DSA_WS_ATTN:
       return dsa::kWsHeaderBytes;
+    case DSA_WS_TOPK:
+      return dsa::kWsHeaderBytes + dsa::topk_cand_bytes(*d);
     case DSA_WS_LAYER:
       return layer_ws(*d, false).total;
     case DSA_WS_DECODE_ATTN:
@@ -278,7 +282,8 @@ dsa_status dsa_topk_select(const dsa_dims* d, const float* scores, int64_t ld,
     cudaError_t e = dsa::launch_key_norm_max(*d, k_idx, h, st);
     if (e != cudaSuccess) return DSA_ERR_CUDA;
   }
-  return from_cuda(dsa::launch_topk(*d, scores, ld, q_idx, k_idx, w_idx, idx, h, st));
+  return from_cuda(dsa::launch_topk(*d, scores, ld, q_idx, k_idx, w_idx, idx, h,
+                                    static_cast<char*>(ws) + dsa::kWsHeaderBytes, st));
 }
 
 dsa_status dsa_sparse_attn_prefill(const dsa_dims* d, const uint16_t* q, const uint16_t* latent,

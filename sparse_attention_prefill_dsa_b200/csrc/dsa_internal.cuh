@@ -81,9 +81,13 @@ cudaError_t launch_quantize_fp8(const uint16_t* x, int64_t rows, int cols, uint8
                                 float* scale, uint16_t* xhat, cudaStream_t st);
 cudaError_t launch_key_norm_max(const dsa_dims& d, const uint16_t* k_idx, WsHeader* ws,
                                 cudaStream_t st);
+// Rows longer than one CTA stages (more than 49,152 keys) are selected in two
+// passes through a candidate buffer of topk_cand_bytes(d) bytes (0 for shorter
+// rows, where `cand` may be null).
+size_t topk_cand_bytes(const dsa_dims& d);
 cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld,
                         const uint16_t* q_idx, const uint16_t* k_idx, const float* w_idx,
-                        int32_t* idx, WsHeader* ws, cudaStream_t st);
+                        int32_t* idx, WsHeader* ws, void* cand, cudaStream_t st);
 // max_s ||[latent_s, rope_s]|| into the header, read by launch_sparse_attn's
 // kernel (launch it first, on the same stream, with the header's field zero).
 cudaError_t launch_attn_key_norm_max(const dsa_dims& d, const uint16_t* latent, const uint16_t* rope,

@@ -7,7 +7,13 @@
 // thread, whose maintainers grant no tie exception between chunkings.
 //
 // One CTA (384 threads) per query row; the row's float32 scores s = 0..t are
-// staged once in shared memory (t + 1 <= 49152 -> at most 192 KB).
+// staged once in shared memory (t + 1 <= 49152 -> at most 192 KB). Longer
+// rows take two levels: pass 1 selects the top-k of every segment of at most
+// 32,768 keys of a row (one CTA per segment), pass 2 the top-k among the
+// segments' winners. The whole row's top-k is a subset of its segments'
+// top-k sets (a key beaten by k keys of its own segment is beaten by them in
+// the row), and both passes use the same exact order, so the result is the
+// one-level selection's.
 //
 // k-th largest value, exactly: a bucket select. The value range [L, U] of the
 // candidates is cut into 2,048 equal buckets, bucket(v) = floor((v - L) * 2048 /
@@ -324,7 +330,7 @@ __device__ bool kth_largest(const float* sc, int n, int k, float vmin, float vma
 template <class Cls>
 __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int32_t* __restrict__ out,
                                int32_t* __restrict__ stage, Cls cls, Scratch& sm, WsHeader* ws, int row,
-                               int a_known = -1) {
+                               int a_known = -1, int key_off = 0, const int32_t* kmap = nullptr) {
   int beg, end;
   my_segment(n, beg, end);
   unsigned int a = 0, t = 0;
@@ -347,7 +353,8 @@ __device__ void emit_selection(const float* sc, int n, int need_ties, int k, int
     bool keep = c == kAbove;
     if (c == kTie) keep = ties_before++ < need_ties;
     if (keep) {
-      if (pos < k) stage[pos] = s;  // never write past the row (a count mismatch is reported below)
+      // never write past the row (a count mismatch is reported below)
+      if (pos < k) stage[pos] = kmap ? __ldg(kmap + s) : s + key_off;
       ++pos;
     }
   });
@@ -456,20 +463,52 @@ struct TopkArgs {
   int bcap;   // band cache capacity (refine only)
   int kst_extra;  // bytes of key staging after cand: kKstExtraBytes (8 re-score warps) or 0 (4)
   int kst_warps;  // warps that re-score band keys (8, or 4 when shared memory is short)
+  // Two-level select for rows longer than one CTA's shared memory holds.
+  // pass 1 takes each row's keys in segments of seg_len and writes every
+  // segment's own top-k (ascending keys) to cand [n_q][n_seg][k]; pass 2
+  // selects each row's top-k among those candidates. Every segment before a
+  // row's last non-empty one holds seg_len >= k keys and gives exactly k
+  // candidates, so a row's candidates are ascending keys with -1 only at the
+  // end, and the (score, key) order among them is the order of positions.
+  // pass 0 is the one-level select.
+  int pass, seg_len, n_seg;
+  int32_t* cand;
 };
 
 template <bool kRefine>
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ Scratch sm;
-  const int row = blockIdx.x;
-  const int t = a.q_pos0 + row;
-  const int n = t + 1;
   const int k = a.k;
-  int32_t* out = a.idx + static_cast<int64_t>(row) * k;
+  int row, n, key_off = 0;
+  const int32_t* kmap = nullptr;  // pass 2: key of each position of the candidate row
+  int32_t* out;
+  if (a.pass == 1) {  // segment seg of the row
+    row = blockIdx.x / a.n_seg;
+    const int seg = blockIdx.x - row * a.n_seg;
+    key_off = seg * a.seg_len;
+    n = min(a.seg_len, a.q_pos0 + row + 1 - key_off);
+    out = a.cand + (static_cast<int64_t>(row) * a.n_seg + seg) * k;
+    if (n <= 0) {  // a segment past the query's position
+      for (int c = threadIdx.x; c < k; c += kThreads) out[c] = -1;
+      return;
+    }
+  } else if (a.pass == 2) {  // the row's candidates
+    row = blockIdx.x;
+    const int t = a.q_pos0 + row;
+    const int nv = t / a.seg_len + 1;  // non-empty segments
+    n = (nv - 1) * k + min(k, t + 1 - (nv - 1) * a.seg_len);
+    kmap = a.cand + static_cast<int64_t>(row) * a.n_seg * k;
+    out = a.idx + static_cast<int64_t>(row) * k;
+  } else {
+    row = blockIdx.x;
+    n = a.q_pos0 + row + 1;
+    out = a.idx + static_cast<int64_t>(row) * k;
+  }
 
-  if (n <= k) {  // every causal key is kept
-    for (int c = threadIdx.x; c < k; c += kThreads) out[c] = c < n ? c : -1;
+  if (n <= k) {  // every key of the row (or segment, or candidate list) is kept
+    for (int c = threadIdx.x; c < k; c += kThreads)
+      out[c] = c < n ? (kmap ? __ldg(kmap + c) : c + key_off) : -1;
     return;
   }
 
@@ -494,8 +533,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   }
 
   // ---- stage the row (and the query's indexer row) with asynchronous copies
-  const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
-  const int n4 = n & ~3;
+  const float* srow = a.scores + static_cast<int64_t>(row) * a.ld + key_off;
+  const int n4 = kmap ? 0 : n & ~3;  // pass 2 gathers its candidates' scores below
   for (int s = threadIdx.x * 4; s < n4; s += kThreads * 4) cp_async16(sc + s, srow + s);
   // the q row, widened to float64 once while the copies fly (only the high
   // words are kept), and this warp's share of A_t = sum_j |w_j| ||q_j||
@@ -542,7 +581,17 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     }
     if (l0 == 0) sm.wd[w0] = acc;
   }
-  for (int s = n4 + threadIdx.x; s < n; s += kThreads) sc[s] = __ldg(srow + s);
+  for (int s = n4 + threadIdx.x; s < n; s += kThreads) {
+    int key = s;
+    if (kmap) {
+      key = __ldg(kmap + s);
+      if (key < 0 || key > a.q_pos0 + row) {  // pass 1 wrote no such candidate
+        report(a.ws, kDevInternal, static_cast<unsigned>(row));
+        key = 0;
+      }
+    }
+    sc[s] = __ldg(srow + key);
+  }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   // canonicalise -0 and find the row's range
@@ -575,12 +624,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   if (!kRefine) {
     emit_selection(
         sc, n, k - n_above, k, out, hist,
-        [&](float v) { return v > vk ? kAbove : (v == vk ? kTie : kBelow); }, sm, a.ws, row);
+        [&](float v) { return v > vk ? kAbove : (v == vk ? kTie : kBelow); }, sm, a.ws, row, -1, key_off, kmap);
     return;
   }
 
   // ---------------- exact float64 order: certified band + float64 re-score
   const int HI = a.HI, DI = a.DI;
+  // the key (cache row) at position s of the staged row
+  auto key_of = [&](int s) { return kmap ? __ldg(kmap + s) : s + key_off; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* p = reinterpret_cast<unsigned char*>(qhi) + kQRowBytes;
   unsigned long long* bx = reinterpret_cast<unsigned long long*>(p);   // band cache
@@ -636,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   if (r == tot_band) {  // the whole band is kept: no re-score needed
     emit_selection(
         sc, n, 0, k, out, hist, [&](float v) { return v >= lo_f ? kAbove : kBelow; }, sm, a.ws, row,
-        c_in + c_band);
+        c_in + c_band, key_off, kmap);
     return;
   }
 
@@ -651,13 +702,13 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     uint2 raw[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)], DI) : make_uint2(0u, 0u);
+      raw[e] = b < tot_band ? load_key_part(a.k_idx, key_of(bidx[min(b + e, tot_band - 1)]), DI) : make_uint2(0u, 0u);
     for (; b < tot_band; b += 4 * kw) {
       const int bn = b + 4 * kw;
       uint2 nraw[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)], DI)
+        nraw[e] = bn < tot_band ? load_key_part(a.k_idx, key_of(bidx[min(bn + e, tot_band - 1)]), DI)
                                 : make_uint2(0u, 0u);
       const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
                                   : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
@@ -696,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     const int kept = c_in + (bk0 >= 0 && sc[bk0] > hi_f) + (bk1 >= 0 && sc[bk1] > hi_f);
     emit_selection(
         sc, n, 0, k, out, hist, [&](float v) { return v > hi_f ? kAbove : kBelow; }, sm, a.ws, row,
-        counted ? kept : -1);
+        counted ? kept : -1, key_off, kmap);
     return;
   }
 
@@ -718,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     for (int jj = warp < kw ? 4 * warp : nb; jj < nb; jj += 4 * kw) {
       uint2 raw[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) raw[e] = load_key_part(a.k_idx, tile_s[min(jj + e, nb - 1)], DI);
+      for (int e = 0; e < 4; ++e) raw[e] = load_key_part(a.k_idx, key_of(tile_s[min(jj + e, nb - 1)]), DI);
       const double xl = DI == 128 ? rescore4<128>(qhi, w_lane, raw, my_kst, HI)
                                   : rescore4<32>(qhi, w_lane, raw, my_kst, HI);
       if (lane < 4 && jj + lane < nb) tile_x[jj + lane] = xl;
@@ -761,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
         if (isnan(v)) return kTie;
         return v > hi_f ? kAbove : kBelow;
       },
-      sm, a.ws, row);
+      sm, a.ws, row, -1, key_off, kmap);
 }
 
 __global__ void key_norm_max_kernel(const uint16_t* __restrict__ k_idx, int T, int DI,
@@ -795,24 +846,31 @@ cudaError_t launch_key_norm_max(const dsa_dims& d, const uint16_t* k_idx, WsHead
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, const uint16_t* q_idx,
-                        const uint16_t* k_idx, const float* w_idx, int32_t* idx, WsHeader* ws,
-                        cudaStream_t st) {
-  TopkArgs a;
-  a.scores = scores;
-  a.ld = ld;
-  a.n_q = d.n_q;
-  a.q_pos0 = d.q_pos0;
-  a.k = d.top_k;
-  a.q_idx = q_idx;
-  a.k_idx = k_idx;
-  a.w_idx = w_idx;
-  a.HI = d.n_idx_heads;
-  a.DI = d.d_idx;
-  a.idx = idx;
-  a.ws = ws;
-  a.n_cap = ((d.q_pos0 + d.n_q) + 3) & ~3;
-  const bool refine = q_idx != nullptr;
+namespace {
+
+// Rows up to kOneLevelRow keys are selected in one pass; longer ones in
+// segments of at most kMaxSegment keys.
+constexpr int kOneLevelRow = 49152;
+constexpr int kMaxSegment = 32768;
+
+struct TwoLevel {
+  int n_seg = 0, seg_len = 0;
+};
+
+TwoLevel two_level(const dsa_dims& d) {
+  TwoLevel t;
+  const int64_t r = static_cast<int64_t>(d.q_pos0) + d.n_q;  // the longest row
+  if (r <= kOneLevelRow) return t;
+  t.n_seg = static_cast<int>((r + kMaxSegment - 1) / kMaxSegment);
+  t.seg_len = static_cast<int>(((r + t.n_seg - 1) / t.n_seg + 3) & ~int64_t{3});
+  return t;
+}
+
+// One launch of topk_kernel over `grid` CTAs with rows of up to `row_cap`
+// staged scores: picks the shared-memory layout (two CTAs per SM with eight
+// re-scoring warps, else one with eight, else one with four) and launches.
+cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStream_t st) {
+  a.n_cap = (row_cap + 3) & ~3;
   int max_smem = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -823,8 +881,7 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   a.kst_warps = kRescoreWarps;
   if (refine) {
     // layout after cand: [key staging extra][q row][band cache (>= the slow
-    // path's scratch)]. Prefer two CTAs per SM with eight re-scoring warps,
-    // then one CTA per SM with eight, then one with four (no extra staging).
+    // path's scratch)]
     bytes += kQRowBytes;
     const size_t min_cache = kSlowScratchBytes > 256 * 12 ? kSlowScratchBytes : 256 * 12;
     const size_t full = static_cast<size_t>(max_smem) - static_bytes;
@@ -857,14 +914,55 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
     e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(bytes));
     if (e != cudaSuccess) return e;
-    topk_kernel<true><<<d.n_q, kThreads, bytes, st>>>(a);
+    topk_kernel<true><<<grid, kThreads, bytes, st>>>(a);
   } else {
     e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(bytes));
     if (e != cudaSuccess) return e;
-    topk_kernel<false><<<d.n_q, kThreads, bytes, st>>>(a);
+    topk_kernel<false><<<grid, kThreads, bytes, st>>>(a);
   }
   return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t topk_cand_bytes(const dsa_dims& d) {
+  const TwoLevel t = two_level(d);
+  return static_cast<size_t>(d.n_q) * t.n_seg * d.top_k * sizeof(int32_t);
+}
+
+cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, const uint16_t* q_idx,
+                        const uint16_t* k_idx, const float* w_idx, int32_t* idx, WsHeader* ws,
+                        void* cand, cudaStream_t st) {
+  TopkArgs a;
+  a.scores = scores;
+  a.ld = ld;
+  a.n_q = d.n_q;
+  a.q_pos0 = d.q_pos0;
+  a.k = d.top_k;
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.w_idx = w_idx;
+  a.HI = d.n_idx_heads;
+  a.DI = d.d_idx;
+  a.idx = idx;
+  a.ws = ws;
+  a.pass = 0;
+  a.seg_len = 0;
+  a.n_seg = 0;
+  a.cand = nullptr;
+  const bool refine = q_idx != nullptr;
+  const TwoLevel t = two_level(d);
+  if (t.n_seg == 0) return launch_pass(a, d.q_pos0 + d.n_q, d.n_q, refine, st);
+  if (!cand) return cudaErrorInvalidValue;
+  a.seg_len = t.seg_len;
+  a.n_seg = t.n_seg;
+  a.cand = static_cast<int32_t*>(cand);
+  a.pass = 1;
+  cudaError_t e = launch_pass(a, t.seg_len, d.n_q * t.n_seg, refine, st);
+  if (e != cudaSuccess) return e;
+  a.pass = 2;
+  return launch_pass(a, t.n_seg * d.top_k, d.n_q, refine, st);
 }
 
 }  // namespace dsa

@@ -80,6 +80,15 @@ def test_workspace_sizes(dsa):
     ld1 = 49152
     layer1 = 256 + ld1 * 4 + (2048 * 4 + 255) // 256 * 256
     assert dsa.dsa_workspace_size(d1, dsa.DSA_WS_DECODE_LAYER) == layer1 + part
+    # rows past 49,152 keys: a top-k candidate buffer of ceil(R / 32768) segments
+    for n_q, q_pos0, T, n_seg in ((1, 49151, 49152, 0), (1, 49152, 49153, 2),
+                                  (1024, 130048, 131072, 4), (64, 65504, 70000, 3)):
+        dl = workloads.make_dims(n_q, q_pos0, T, 32, 512, 64, 32, 128, 2048)
+        cand = n_q * n_seg * 2048 * 4
+        assert dsa.dsa_workspace_size(dl, dsa.DSA_WS_TOPK) == 256 + cand
+        ldl = (T + 127) // 128 * 128
+        assert dsa.dsa_workspace_size(dl, dsa.DSA_WS_LAYER) == \
+            256 + n_q * ldl * 4 + n_q * 2048 * 4 + cand
 
 
 FAKE = 1 << 20  # an aligned, never dereferenced address
@@ -104,7 +113,7 @@ def test_host_validation_before_any_device_call(dsa):
     bad = dsa.make_dims(d)
     bad.n_q = d.n_q + 1
     assert _layer(dsa, bad) == dsa.DSA_ERR_CAUSAL
-    for field, val in (("top_k", 0), ("top_k", 2049), ("ctx_len", 49153), ("n_heads", 8),
+    for field, val in (("top_k", 0), ("top_k", 2049), ("ctx_len", 131073), ("n_heads", 8),
                        ("d_latent", 256), ("n_idx_heads", 64), ("flags", 4), ("n_q", -1),
                        ("softmax_scale", 0.0)):
         bad = dsa.make_dims(d)
