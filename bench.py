@@ -303,7 +303,7 @@ def run_ours(args):
     else:
         torch.cuda.set_device(local)
     dsa.library()
-    wl = workloads.BY_NAME[args.workload]
+    wl = workloads.ALL_BY_NAME[args.workload]
     d = wl.dims
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     x = workloads.generate(d, rank_seed(wl.seed, rank), wl.kind, w_mode)
@@ -366,7 +366,11 @@ def run_ours(args):
     # ---- per-kernel durations, same inputs and launch configuration
     ld = (d.ctx_len + 127) // 128 * 128
     scores = torch.empty(d.n_q, ld, dtype=torch.float32, device="cuda")
-    ws_small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    # one workspace for the three single-step calls: the largest they need (the
+    # top-k's candidate buffer on rows past 49,152 keys)
+    ws_small = torch.empty(max(dsa.dsa_workspace_size(d, w) for w in
+                               (dsa.DSA_WS_INDEX_SCORES, dsa.DSA_WS_TOPK, dsa.DSA_WS_ATTN)),
+                           dtype=torch.uint8, device="cuda")
     names = ("index_scores", "topk_select", "sparse_attn")
     d1 = dataclasses.replace(d, flags=0)  # the single-step calls take no flag
     if args.fp8_indexer:
@@ -539,7 +543,7 @@ def run_split(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dsa.library()
-    wl = workloads.BY_NAME[args.workload]
+    wl = workloads.ALL_BY_NAME[args.workload]
     d = wl.dims
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     x = workloads.generate(d, wl.seed, wl.kind, w_mode)  # one chunk, the same on every rank
@@ -676,7 +680,7 @@ def run_reference(args):
     import oracle
 
     oracle.build()
-    wl = workloads.BY_NAME[args.workload]
+    wl = workloads.ALL_BY_NAME[args.workload]
     d = wl.dims
     w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     x = workloads.generate(d, wl.seed, wl.kind, w_mode)
@@ -711,7 +715,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="chunk8k_ctx17k", choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--workload", default="chunk8k_ctx17k", choices=sorted(workloads.ALL_BY_NAME))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="query rows of the bounded CPU-oracle sample (0: about 12 s of work)")

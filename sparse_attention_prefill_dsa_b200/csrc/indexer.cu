@@ -347,18 +347,33 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI, FP8>::kThreads, 1)
         // FP8: the key row's scale, applied to the finished head sum (a power
         // of two: relu(s_k x) = s_k relu(x), and the product is exact)
         const float ks = FP8 ? (s < p.ctx_len ? __ldg(p.k_scale + s) : 0.f) : 1.f;
-        // two 32-column groups per TMEM wait; the weights of a group are read
-        // as float4 broadcasts
-#pragma unroll 1
+        // four 32-column groups, two per TMEM wait; with 32 heads the loads of
+        // the next two groups are in flight while the current two are summed
+        // (with 2 heads a group holds 16 queries and the registers would not
+        // hold four). The weights of a group are read as float4 broadcasts.
+        constexpr bool kAhead = HI == 32;
+        uint32_t v[4][32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + h * 32, v[h]);
+        tmem_ld_wait();
+#pragma unroll
         for (int g2 = 0; g2 < 2; ++g2) {
-          uint32_t v[2][32];
+          if (g2 == 0 && kAhead) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + (2 * g2 + h) * 32, v[h]);
-          tmem_ld_wait();
+            for (int h = 2; h < 4; ++h)
+              tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + h * 32, v[h]);
+          } else if (g2 == 1) {
+            if (!kAhead) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int col0 = wg * 128 + (2 * g2 + h) * 32;
+              for (int h = 2; h < 4; ++h)
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + h * 32, v[h]);
+            }
+            tmem_ld_wait();
+          }
+#pragma unroll
+          for (int h = 2 * g2; h < 2 * g2 + 2; ++h) {
+            const int col0 = wg * 128 + h * 32;
             float wv[32];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -370,10 +385,19 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI, FP8>::kThreads, 1)
             }
 #pragma unroll
             for (int qq = 0; qq < 32 / HI; ++qq) {
-              float acc = 0.f;
+              // the head sum in four interleaved partial sums (heads j mod 4),
+              // so that consecutive multiply-adds do not wait on each other
+              constexpr int kPart = HI >= 4 ? 4 : HI;
+              float part[kPart];
+#pragma unroll
+              for (int u = 0; u < kPart; ++u) part[u] = 0.f;
 #pragma unroll
               for (int j = 0; j < HI; ++j)
-                acc = fmaf(wv[qq * HI + j], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f), acc);
+                part[j % kPart] = fmaf(wv[qq * HI + j], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f),
+                                       part[j % kPart]);
+              float acc = part[0];
+#pragma unroll
+              for (int u = 1; u < kPart; ++u) acc += part[u];
               const int i = qb * C::kQB + (col0 + qq * HI) / HI;
               if (i < p.n_q && s <= p.q_pos0 + i && DSA_IN_BOUNDS(p.ws, s, p.ld, 20))
                 p.scores[static_cast<int64_t>(i) * p.ld + s] = FP8 ? acc * ks : acc;

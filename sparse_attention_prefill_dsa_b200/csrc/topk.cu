@@ -475,7 +475,10 @@ struct TopkArgs {
   int32_t* cand;
 };
 
-template <bool kRefine>
+// kPass: 0 the one-level select, 1 and 2 the two passes of the long-row
+// select (a template parameter, so that the one-level kernel carries none of
+// the other passes' key mapping)
+template <bool kRefine, int kPass>
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ Scratch sm;
@@ -483,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   int row, n, key_off = 0;
   const int32_t* kmap = nullptr;  // pass 2: key of each position of the candidate row
   int32_t* out;
-  if (a.pass == 1) {  // segment seg of the row
+  if (kPass == 1) {  // segment seg of the row
     row = blockIdx.x / a.n_seg;
     const int seg = blockIdx.x - row * a.n_seg;
     key_off = seg * a.seg_len;
@@ -493,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       for (int c = threadIdx.x; c < k; c += kThreads) out[c] = -1;
       return;
     }
-  } else if (a.pass == 2) {  // the row's candidates
+  } else if (kPass == 2) {  // the row's candidates
     row = blockIdx.x;
     const int t = a.q_pos0 + row;
     const int nv = t / a.seg_len + 1;  // non-empty segments
@@ -866,6 +869,27 @@ TwoLevel two_level(const dsa_dims& d) {
   return t;
 }
 
+template <bool kRefine, int kPass>
+cudaError_t launch_instance(const TopkArgs& a, int grid, size_t bytes, cudaStream_t st) {
+  const cudaError_t e = cudaFuncSetAttribute(topk_kernel<kRefine, kPass>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  topk_kernel<kRefine, kPass><<<grid, kThreads, bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kernel(const TopkArgs& a, int grid, size_t bytes, bool refine, cudaStream_t st) {
+  switch (a.pass * 2 + (refine ? 1 : 0)) {
+    case 0: return launch_instance<false, 0>(a, grid, bytes, st);
+    case 1: return launch_instance<true, 0>(a, grid, bytes, st);
+    case 2: return launch_instance<false, 1>(a, grid, bytes, st);
+    case 3: return launch_instance<true, 1>(a, grid, bytes, st);
+    case 4: return launch_instance<false, 2>(a, grid, bytes, st);
+    default: return launch_instance<true, 2>(a, grid, bytes, st);
+  }
+}
+
 // One launch of topk_kernel over `grid` CTAs with rows of up to `row_cap`
 // staged scores: picks the shared-memory layout (two CTAs per SM with eight
 // re-scoring warps, else one with eight, else one with four) and launches.
@@ -909,19 +933,7 @@ cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStre
   } else if (static_cast<size_t>(max_smem) < bytes + static_bytes) {
     return cudaErrorInvalidConfiguration;
   }
-  cudaError_t e;
-  if (refine) {
-    e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bytes));
-    if (e != cudaSuccess) return e;
-    topk_kernel<true><<<grid, kThreads, bytes, st>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bytes));
-    if (e != cudaSuccess) return e;
-    topk_kernel<false><<<grid, kThreads, bytes, st>>>(a);
-  }
-  return cudaGetLastError();
+  return launch_kernel(a, grid, bytes, refine, st);
 }
 
 }  // namespace

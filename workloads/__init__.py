@@ -78,6 +78,15 @@ WORKLOADS = [
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
+# A longer context than the five workloads above reach: rows of more than
+# 49,152 keys, which the top-k selects in two passes. Timed by the bench
+# (--workload); the parity tests cover such rows with their own smaller chunks.
+LONG_WORKLOADS = [
+    Workload("chunk4k_ctx128k", make_dims(4096, 126976, 131072, 32, 512, 64, 32, 128, 2048), 5,
+             "normal", "4,096-query chunk at 126,976..131,071 of a 131,072 context, k=2048"),
+]
+ALL_BY_NAME = {**BY_NAME, **{w.name: w for w in LONG_WORKLOADS}}
+
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """float32 -> bf16 bit patterns (uint16), round to nearest even. Finite inputs."""
@@ -134,7 +143,7 @@ def generate(d: Dims, seed: int, kind: str = "normal", w_mode: str = "uniform") 
 
 
 def workload_inputs(name: str, w_mode: str | None = None) -> tuple[Dims, dict]:
-    wl = BY_NAME[name]
+    wl = ALL_BY_NAME[name]
     if w_mode is None:
         w_mode = "ones" if wl.kind == "ternary_ties" else "uniform"
     return wl.dims, generate(wl.dims, wl.seed, wl.kind, w_mode)
