@@ -461,6 +461,31 @@ def run_ours(args):
     dsa.check(dsa.dsa_device_status(ws_layer, stream=stream))
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     barrier(world)
+    # the copies alone, as the bound of the end-to-end figure: every input in
+    # (one copy per tensor, pinned host memory) and the output back, each
+    # direction by itself, median of the steps
+    def copy_ms(h2d_on, d2h_on):
+        ts = []
+        for _ in range(max(3, args.steps)):
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            joined = torch.cuda.Event()
+            c0.record(e2e_streams[0])
+            e2e_streams[2].wait_event(c0)
+            if h2d_on:
+                with torch.cuda.stream(e2e_streams[0]):
+                    for k_, v_ in pinned.items():
+                        dev_tensors[k_].copy_(v_, non_blocking=True)
+            if d2h_on:
+                with torch.cuda.stream(e2e_streams[2]):
+                    out_host.copy_(out, non_blocking=True)
+            joined.record(e2e_streams[2])
+            e2e_streams[0].wait_event(joined)
+            c1.record(e2e_streams[0])
+            torch.cuda.synchronize()
+            ts.append(c0.elapsed_time(c1))
+        return max_over_ranks(statistics.median(ts), world)
+    h2d_only_ms, d2h_only_ms = copy_ms(True, False), copy_ms(False, True)
+    both_ms = copy_ms(True, True)  # both directions at once, as in the end-to-end call
 
     # the dominant kernel's roofline, with its DRAM traffic when a capture of
     # the current kernel on this workload exists
@@ -499,7 +524,8 @@ def run_ours(args):
                    "indexer": "fp8 (e4m3) variant" if args.fp8_indexer else "bf16",
                    "l2": "flushed: 256 MB write between timed steps"},
         "tflops": tflops,
-        "pct_of_measured_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "bf16_peak": {"tflops": peaks["bf16_tflops"], "source": peaks_src},
         "pct_of_spec_bf16_peak": 100.0 * tflops / SPEC_BF16_TFLOPS,
         "useful_flop_per_step": fl["total"],
         "ms_per_step_median": max_over_ranks(statistics.median(step_ms), world),
@@ -511,6 +537,8 @@ def run_ours(args):
         "e2e": {"value": whole_job_rate(world, d.n_q, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "call": "dsa_prefill_layer_host", "sub_chunks": n_best,
+                "h2d_alone_ms": h2d_only_ms, "d2h_alone_ms": d2h_only_ms,
+                "h2d_and_d2h_together_ms": both_ms,
                 "warmup_ms_by_sub_chunks": {str(k): round(v, 3) for k, v in tried.items()}},
         "gpu_launches": (KERNELS_PER_LAYER + (2 if args.fp8_indexer else 0)) * args.steps,
         "roofline": roof,
@@ -631,7 +659,7 @@ def run_split(args):
                    "top_k": d.top_k, "parallelism": f"query split over {world} ranks "
                    "(cache rows and outputs all-gathered over NCCL)",
                    "ranges": ranges, "l2": "flushed: 256 MB write between timed steps"},
-        "tflops": tflops, "pct_of_measured_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
         "e2e": {"value": d.n_q / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": KERNELS_PER_LAYER * args.steps,
