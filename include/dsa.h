@@ -74,6 +74,13 @@ typedef struct dsa_dims {
  * decode calls ignore it. Outputs agree with the one-SM kernel within
  * rounding; selections are unaffected. */
 #define DSA_FLAG_ATTN_PAIR 2u
+/* dims.flags: dsa_prefill_layer_host does not order itself after the work
+ * that earlier calls left on its streams; the caller orders it instead. With
+ * two sets of device tensors used in turn, each set reused only after an
+ * event recorded on streams[2] at the end of the call that last used it,
+ * the copy-in of one chunk then overlaps the layers and the copy-out of the
+ * previous one. The other calls reject it (DSA_ERR_DIMS). */
+#define DSA_FLAG_HOST_UNORDERED 4u
 
 /* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):
  *   (n_heads, d_latent, d_rope)  in {(4, 64, 16), (32, 512, 64)}
@@ -304,7 +311,11 @@ typedef struct {
  * The outputs are complete once streams[2] has finished the work this call
  * enqueued; the device status of the layer calls is read with
  * dsa_device_status(workspace, streams[1]). Results are bit-identical to one
- * dsa_prefill_layer call on the whole chunk.
+ * dsa_prefill_layer call on the whole chunk. Unless dims.flags holds
+ * DSA_FLAG_HOST_UNORDERED, the call first orders its copies after the layers
+ * and its layers after the copy-outs that earlier calls left on the streams,
+ * so that back-to-back calls on the same device tensors never overwrite a
+ * buffer still in use.
  * Errors: those of dsa_prefill_layer, DSA_ERR_NULL for a missing stream,
  * event or device tensor, DSA_ERR_DIMS for n_sub < 1. */
 dsa_status dsa_prefill_layer_host(const dsa_dims* dims, const uint16_t* q, const uint16_t* latent,

@@ -422,7 +422,8 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const ui
                                   const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                                   const dsa_device_tensors* dev, void* ws, size_t ws_bytes,
                                   void* const streams[3], void* const events[2], int32_t n_sub) {
-  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR);
+  dsa_status s =
+      check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR | DSA_FLAG_HOST_UNORDERED);
   if (s != DSA_OK) return s;
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out || !dev || !streams || !events)
     return DSA_ERR_NULL;
@@ -445,12 +446,15 @@ dsa_status dsa_prefill_layer_host(const dsa_dims* d, const uint16_t* q, const ui
   cudaEvent_t ev_b = static_cast<cudaEvent_t>(events[1]);
   // work already on the streams (an earlier call) ends before this call's
   // copies overwrite the inputs its layers read and its layers overwrite the
-  // outputs its copies read
-  cudaError_t e = cudaEventRecord(ev_a, s_run);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_a, 0);
-  if (e == cudaSuccess) e = cudaEventRecord(ev_b, s_out);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_run, ev_b, 0);
-  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  // outputs its copies read (unless the caller orders the calls itself)
+  cudaError_t e = cudaSuccess;
+  if ((d->flags & DSA_FLAG_HOST_UNORDERED) == 0u) {
+    e = cudaEventRecord(ev_a, s_run);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_a, 0);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_b, s_out);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_run, ev_b, 0);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+  }
   if ((s = clear_header(ws, s_run)) != DSA_OK) return s;  // once: sub-chunks keep each other's status
   if (d->n_q == 0) return DSA_OK;
   const size_t T = static_cast<size_t>(d->ctx_len);

@@ -271,6 +271,61 @@ def test_host_entry_matches_device_entry(dsa, n_q, n_sub):
     assert np.array_equal(idx_h.numpy(), idx_ref)
 
 
+def test_host_entry_unordered_calls_alternating_buffers(dsa):
+    """DSA_FLAG_HOST_UNORDERED: four back-to-back host calls on two chunks,
+    alternating two sets of device tensors (each reused after an event at the
+    end of the call that last used it), overlap one call's copy-in with the
+    previous call's layers; every call's outputs keep the bits of
+    dsa_prefill_layer on its own chunk."""
+    import dataclasses
+
+    import torch
+
+    chunks = []
+    for n_q, seed_shift in ((96, 0), (133, 1)):
+        d, x = _reduced("chunk2k_ctx8k", n_q)
+        if seed_shift:  # a second chunk with other inputs of another length
+            x = workloads.generate(d, 977, "normal", "uniform")
+        xd = stage(x)
+        chunks.append((d, {k: v.cpu().pin_memory() for k, v in xd.items()}, run_layer(dsa, d, xd)))
+    d_max = max((c[0] for c in chunks), key=lambda d_: d_.n_q)
+    sets = []
+    for _ in range(2):
+        dev_t = {k: torch.empty(d_max.ctx_len if k in ("latent", "rope", "k_idx") else d_max.n_q,
+                                *v.shape[1:], dtype=v.dtype, device="cuda")
+                 for k, v in chunks[1][1].items()}
+        dev_t["out"] = empty_bf16(d_max.n_q, d_max.n_heads, d_max.d_latent)
+        sets.append(dev_t)
+    streams = (torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream())
+    events = (torch.cuda.Event(), torch.cuda.Event())
+    free = [torch.cuda.Event(), torch.cuda.Event()]
+    for ev in (*events, *free):
+        ev.record()
+    ws = workspace(dsa.dsa_workspace_size(d_max, dsa.DSA_WS_LAYER))
+    outs = []
+    for call in range(4):
+        d, pinned, _ = chunks[call % 2]
+        b = call % 2
+        streams[0].wait_event(free[b])
+        streams[1].wait_event(free[b])
+        out_h = torch.empty(d.n_q, d.n_heads, d.d_latent, dtype=torch.bfloat16).pin_memory()
+        dh = dataclasses.replace(d, flags=dsa.DSA_FLAG_HOST_UNORDERED)
+        dsa.check(dsa.dsa_prefill_layer_host(dh, pinned["q"], pinned["latent"], pinned["rope"],
+                                             pinned["q_idx"], pinned["k_idx"], pinned["w_idx"],
+                                             out_h, None, None, sets[b], ws, streams, events, 8))
+        free[b].record(streams[2])
+        outs.append(out_h)
+    torch.cuda.synchronize()
+    dsa.check(dsa.dsa_device_status(ws, stream=streams[1]))
+    for call, out_h in enumerate(outs):
+        assert np.array_equal(host_bf16_as_f32(out_h), chunks[call % 2][2][0]), call
+    # the flag belongs to the host call alone
+    d0 = dataclasses.replace(chunks[0][0], flags=dsa.DSA_FLAG_HOST_UNORDERED)
+    assert dsa.dsa_prefill_layer(d0, *[chunks[0][1][k].cuda() for k in
+                                       ("q", "latent", "rope", "q_idx", "k_idx", "w_idx")],
+                                 sets[0]["out"], None, None, ws) == dsa.DSA_ERR_DIMS
+
+
 def test_sparse_attn_entry_point_on_given_sets(dsa, oracle_lib):
     """dsa_sparse_attn_prefill on oracle-chosen sets, with padding and shuffled order."""
     import torch
