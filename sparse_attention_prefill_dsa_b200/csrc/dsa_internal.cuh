@@ -15,7 +15,8 @@ struct WsHeader {
   unsigned long long kmax_bits;  // float64 bit pattern of max_s ||k_idx[s]||_2 (>= 0)
   unsigned int akmax_bits;       // float32 bit pattern of max_s ||[latent_s, rope_s]||_2 (>= 0)
   unsigned int unit_next;        // the indexer's work queue: next unit to hand out
-  unsigned char pad[232];
+  unsigned int topk_redo;        // rows the top-k's window select handed to the bucket select
+  unsigned char pad[228];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 

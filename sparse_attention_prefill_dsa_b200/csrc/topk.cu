@@ -58,6 +58,8 @@ namespace dsa {
 namespace {
 
 constexpr int kThreads = 384;
+// first index of a row the window select hands back to topk_kernel
+constexpr int32_t kRedoMarker = static_cast<int32_t>(0x80000000u);
 constexpr int kWarps = kThreads / 32;
 constexpr int kRescoreWarps = 8;  // warps that re-score band keys (their staging fits hist + cand + extra)
 constexpr int kBins = 2048;
@@ -111,6 +113,7 @@ __device__ __forceinline__ unsigned long long d2key(double x) {
 
 // ------------------------------------------------------------ block helpers
 
+template <int NT = kThreads>
 __device__ __forceinline__ void block_minmax(float& mn, float& mx, Scratch& sc) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -126,7 +129,7 @@ __device__ __forceinline__ void block_minmax(float& mn, float& mx, Scratch& sc) 
   mn = sc.wf0[0];
   mx = sc.wf1[0];
 #pragma unroll
-  for (int w = 1; w < kWarps; ++w) {
+  for (int w = 1; w < NT / 32; ++w) {
     mn = fminf(mn, sc.wf0[w]);
     mx = fmaxf(mx, sc.wf1[w]);
   }
@@ -134,6 +137,7 @@ __device__ __forceinline__ void block_minmax(float& mn, float& mx, Scratch& sc) 
 }
 
 // Exclusive prefix sum of a packed pair of 32-bit counters; *total gets the sum.
+template <int NT = kThreads>
 __device__ __forceinline__ unsigned long long block_excl_scan64(unsigned long long v,
                                                                 unsigned long long* total,
                                                                 Scratch& sc) {
@@ -148,7 +152,7 @@ __device__ __forceinline__ unsigned long long block_excl_scan64(unsigned long lo
   __syncthreads();
   unsigned long long base = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     const unsigned long long t = sc.w64[w];
     if (w < warp) base += t;
     tot += t;
@@ -159,9 +163,9 @@ __device__ __forceinline__ unsigned long long block_excl_scan64(unsigned long lo
 }
 
 // hist[0..NB) counts; finds bin b with sum(hist[b+1..]) < kr <= sum(hist[b..]).
-template <int NB>
+template <int NB, int NT = kThreads>
 __device__ int find_bin_from_top(const int* hist, int kr, int* above, Scratch& sc) {
-  constexpr int per = (NB + kThreads - 1) / kThreads;  // bins per thread, counted from the top
+  constexpr int per = (NB + NT - 1) / NT;  // bins per thread, counted from the top
   const int r0 = threadIdx.x * per;
   int local = 0;
 #pragma unroll
@@ -169,7 +173,7 @@ __device__ int find_bin_from_top(const int* hist, int kr, int* above, Scratch& s
     if (r0 + e < NB) local += hist[NB - 1 - (r0 + e)];
   unsigned long long tot;
   const int before =
-      static_cast<int>(block_excl_scan64(static_cast<unsigned long long>(local), &tot, sc));
+      static_cast<int>(block_excl_scan64<NT>(static_cast<unsigned long long>(local), &tot, sc));
   if (before < kr && before + local >= kr) {
     int acc = before;
     for (int e = 0; e < per && r0 + e < NB; ++e) {
@@ -473,6 +477,11 @@ struct TopkArgs {
   // pass 0 is the one-level select.
   int pass, seg_len, n_seg;
   int32_t* cand;
+  // the window select (topk_window_kernel): shared-memory sizes of its chunk
+  // counts and kept-key bitmap; only_marked makes topk_kernel redo only the
+  // rows the window select handed back
+  int fw_chunks, fw_words;
+  int only_marked;
 };
 
 // kPass: 0 the one-level select, 1 and 2 the two passes of the long-row
@@ -507,6 +516,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     row = blockIdx.x;
     n = a.q_pos0 + row + 1;
     out = a.idx + static_cast<int64_t>(row) * k;
+    if (a.only_marked) {  // redo only the rows the window select handed back
+      if (*reinterpret_cast<volatile unsigned int*>(&a.ws->topk_redo) == 0u) return;
+      if (*reinterpret_cast<volatile int32_t*>(out) != kRedoMarker) return;
+    }
   }
 
   if (n <= k) {  // every key of the row (or segment, or candidate list) is kept
@@ -818,6 +831,364 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       sm, a.ws, row, -1, key_off, kmap);
 }
 
+// ---------------------------------------------------------------------------
+// The one-level exact select without the row in shared memory: the window
+// select. One CTA of 192 threads per row and about 50 KB of shared memory, so
+// four rows share an SM (topk_kernel, which stages the row, fits two). The
+// row is read from global memory (from L2 after its first pass) in coalesced
+// chunks of 128 keys, a warp per chunk:
+//   1. the row's range [L, U];
+//   2. a histogram over 2,048 buckets of the range, and the bucket b* that
+//      holds the k-th largest float score v;
+//   3. the window pass: per chunk the number of keys above a window around
+//      b* widened by 2 delta on either side (delta as in topk_kernel), and
+//      the window's keys collected with their scores. Every key within
+//      2 delta of v is in the window, so v, the keys certainly kept
+//      (above v + 2 delta) and the band [v - 2 delta, v + 2 delta] follow from
+//      the window alone;
+//   4. the band re-scored in float64 in the contract's order and ranked by
+//      (X desc, key asc), exactly as in topk_kernel; the window's kept keys
+//      are marked in a bitmap and counted in their chunks;
+//   5. the emit: a scan of the chunk counts places each chunk's kept keys
+//      (the keys above the window and the marked ones) in ascending order.
+// A row whose range is a single value or too wide for a float bucket scale,
+// or whose window holds more than kWinCap keys (heavy ties), is handed back:
+// its first index is set to kRedoMarker and counted in the workspace header,
+// and a second launch of topk_kernel redoes those rows alone.
+constexpr int kFThreads = 192;
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kFChunk = 128;
+constexpr int kWinCap = 256;
+
+template <int DI>
+__global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ Scratch sm;
+  __shared__ int s_ncand, s_chi;
+  const int k = a.k;
+  const int row = blockIdx.x;
+  const int n = a.q_pos0 + row + 1;
+  int32_t* out = a.idx + static_cast<int64_t>(row) * k;
+  if (n <= k) {  // every causal key is kept
+    for (int c = threadIdx.x; c < k; c += kFThreads) out[c] = c < n ? c : -1;
+    return;
+  }
+  const int HI = a.HI;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_chunks = (n + kFChunk - 1) / kFChunk;
+  // shared memory: hist (later the emit's staging) | key staging of the
+  // re-score | q row (float64 high words) | band cache | chunk counts |
+  // kept-key bitmap | window keys and scores
+  int* hist = reinterpret_cast<int*>(smem);
+  uint32_t* kst_all = reinterpret_cast<uint32_t*>(smem + kBins * 4);
+  uint32_t* qhi = kst_all + kFWarps * 512;
+  unsigned long long* bx = reinterpret_cast<unsigned long long*>(
+      reinterpret_cast<unsigned char*>(qhi) + kQRowBytes);
+  int* bidx = reinterpret_cast<int*>(bx + kWinCap);
+  int* chunk_cnt = bidx + kWinCap;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(chunk_cnt + a.fw_chunks);
+  int* cand_pos = reinterpret_cast<int*>(bits + a.fw_words);
+  float* cand_val = reinterpret_cast<float*>(cand_pos + kWinCap);
+  const int qstride = DI + 4;
+
+  const float w_pre = lane < HI ? __ldg(a.w_idx + static_cast<int64_t>(row) * HI + lane) : 0.f;
+  const unsigned long long kmax_bits = *reinterpret_cast<volatile unsigned long long*>(&a.ws->kmax_bits);
+  for (int b = threadIdx.x; b < kBins; b += kFThreads) hist[b] = 0;
+  for (int c = threadIdx.x; c < n_chunks; c += kFThreads) chunk_cnt[c] = 0;
+  for (int w = threadIdx.x; w < (n + 31) / 32; w += kFThreads) bits[w] = 0u;
+  if (threadIdx.x == 0) {
+    s_ncand = 0;
+    s_chi = 0;
+  }
+  // the q row widened to float64 high words, and this warp's share of
+  // A_t = sum_j |w_j| ||q_j|| (heads warp, warp + 6, ...)
+  {
+    constexpr int kHeadsPerWarp = (32 + kFWarps - 1) / kFWarps;
+    const int wpr = DI / 2;
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(a.q_idx + static_cast<int64_t>(row) * HI * DI);
+    uint32_t qv[kHeadsPerWarp][2];
+#pragma unroll
+    for (int u = 0; u < kHeadsPerWarp; ++u) {
+      const int j = warp + u * kFWarps;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int pr = lane + 32 * t;
+        qv[u][t] = (j < HI && pr < wpr) ? __ldg(q32 + j * wpr + pr) : 0u;
+      }
+    }
+    double acc = 0.0;
+#pragma unroll
+    for (int u = 0; u < kHeadsPerWarp; ++u) {
+      const int j = warp + u * kFWarps;
+      double ss = 0.0;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int pr = lane + 32 * t;
+        if (j < HI && pr < wpr && DSA_IN_BOUNDS(a.ws, j * qstride + 2 * pr + 1, kQRowBytes / 4, 50)) {
+          const uint32_t v = qv[u][t];
+          const double lo = static_cast<double>(__uint_as_float(v << 16));
+          const double hi = static_cast<double>(__uint_as_float(v & 0xFFFF0000u));
+          qhi[j * qstride + 2 * pr] = static_cast<uint32_t>(__double2hiint(lo));
+          qhi[j * qstride + 2 * pr + 1] = static_cast<uint32_t>(__double2hiint(hi));
+          ss += lo * lo;
+          ss += hi * hi;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float wj = __shfl_sync(0xffffffffu, w_pre, j & 31);
+      if (j < HI) acc += fabs(static_cast<double>(wj)) * sqrt(ss);
+    }
+    if (lane == 0) sm.wd[warp] = acc;
+  }
+
+  // ---- 1. the row's range
+  const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
+  const float4* s4 = reinterpret_cast<const float4*>(srow);
+  const int n4 = n >> 2;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int i = threadIdx.x; i < n4; i += kFThreads) {
+    const float4 v = __ldg(s4 + i);
+    mn = fminf(fminf(mn, v.x), fminf(fminf(v.y, v.z), v.w));
+    mx = fmaxf(fmaxf(mx, v.x), fmaxf(fmaxf(v.y, v.z), v.w));
+  }
+  for (int s = 4 * n4 + threadIdx.x; s < n; s += kFThreads) {
+    const float v = __ldg(srow + s);
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  block_minmax<kFThreads>(mn, mx, sm);  // (also orders the zeroing above before its use)
+  double A = 0.0;
+  for (int w = 0; w < kFWarps; ++w) A += sm.wd[w];
+  A *= kNormSlack;
+  const double delta = kBoundRel * A * __longlong_as_double(static_cast<long long>(kmax_bits));
+  const Bucketer bucket(mn, mx);
+  bool redo = !(mn < mx) || !bucket.wide || !(delta < 1e30);
+
+  float whi_f = 0.f, lo_f = 0.f, hi_f = 0.f;
+  int c_hi_tot = 0;
+  if (!redo) {
+    // ---- 2. histogram and the bucket of the k-th largest
+    for (int i = threadIdx.x; i < n4; i += kFThreads) {
+      const float4 v = __ldg(s4 + i);
+      atomicAdd(&hist[bucket(v.x)], 1);
+      atomicAdd(&hist[bucket(v.y)], 1);
+      atomicAdd(&hist[bucket(v.z)], 1);
+      atomicAdd(&hist[bucket(v.w)], 1);
+    }
+    for (int s = 4 * n4 + threadIdx.x; s < n; s += kFThreads) atomicAdd(&hist[bucket(__ldg(srow + s))], 1);
+    __syncthreads();
+    int ab;
+    const int bstar = find_bin_from_top<kBins, kFThreads>(hist, k, &ab, sm);
+    // a value in bucket b lies within (b +- 0.5) bucket widths of L up to
+    // float rounding (relative 2^-21 of at most 2048 widths); the window
+    // allows 1.5 widths and 2 delta on either side
+    const double width = (static_cast<double>(mx) - static_cast<double>(mn)) / kBins;
+    const float wlo_f = __double2float_rd(static_cast<double>(mn) + (bstar - 1.5) * width - 2.0 * delta);
+    whi_f = __double2float_ru(static_cast<double>(mn) + (bstar + 1.5) * width + 2.0 * delta);
+
+    // ---- 3. the window pass
+    int c_hi = 0;
+    for (int c = warp; c < n_chunks; c += kFWarps) {
+      const int s0 = c * kFChunk + 4 * lane;
+      float v[4];
+      if (s0 + 3 < n) {
+        const float4 f4 = __ldg(reinterpret_cast<const float4*>(srow + s0));
+        v[0] = f4.x; v[1] = f4.y; v[2] = f4.z; v[3] = f4.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = s0 + e < n ? __ldg(srow + s0 + e) : -INFINITY;
+      }
+      int above = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float f = v[e];
+        above += f > whi_f;
+        if (s0 + e < n && f >= wlo_f && f <= whi_f) {
+          const int pos = atomicAdd(&s_ncand, 1);
+          if (pos < kWinCap) {
+            cand_pos[pos] = s0 + e;
+            cand_val[pos] = f;
+          }
+        }
+      }
+      above = __reduce_add_sync(0xffffffffu, above);
+      if (lane == 0 && DSA_IN_BOUNDS(a.ws, c, a.fw_chunks, 51)) chunk_cnt[c] = above;
+      c_hi += above;
+    }
+    if (lane == 0) atomicAdd(&s_chi, c_hi);
+    __syncthreads();
+    const int n_cand = s_ncand;
+    c_hi_tot = s_chi;
+    redo = !(n_cand <= kWinCap && c_hi_tot < k && c_hi_tot + n_cand >= k);
+    if (!redo) {
+      // ---- 4. v, the certainly kept keys and the band, from the window
+      const int kr = k - c_hi_tot;
+      for (int i = threadIdx.x; i < n_cand; i += kFThreads) {
+        const float vi = cand_val[i];
+        int gt = 0, ge = 0;
+        for (int o = 0; o < n_cand; ++o) {
+          const float u = cand_val[o];
+          gt += u > vi;
+          ge += u >= vi;
+        }
+        if (gt < kr && kr <= ge) sm.bf[0] = vi;
+      }
+      __syncthreads();
+      const float vk = sm.bf[0];
+      lo_f = __double2float_ru(static_cast<double>(vk) - 2.0 * delta);
+      hi_f = __double2float_rd(static_cast<double>(vk) + 2.0 * delta);
+      if (warp == 0) {  // kept above hi_f; the band in window order
+        int nb = 0, nin = 0;
+        for (int i0 = 0; i0 < n_cand; i0 += 32) {
+          const int i = i0 + lane;
+          const bool valid = i < n_cand;
+          const int s2 = valid ? cand_pos[i] : 0;
+          const float f = valid ? cand_val[i] : 0.f;
+          const bool in_band = valid && f >= lo_f && f <= hi_f;
+          const bool above2 = valid && f > hi_f;
+          const unsigned mb = __ballot_sync(0xffffffffu, in_band);
+          nin += __popc(__ballot_sync(0xffffffffu, above2));
+          if (in_band) bidx[nb + __popc(mb & ((1u << lane) - 1u))] = s2;
+          if (above2) {
+            atomicOr(&bits[s2 >> 5], 1u << (s2 & 31));
+            atomicAdd(&chunk_cnt[s2 / kFChunk], 1);
+          }
+          nb += __popc(mb);
+        }
+        if (lane == 0) {
+          sm.bc[0] = nb;
+          sm.bc[1] = nin;
+        }
+      }
+      __syncthreads();
+      const int tot_band = sm.bc[0];
+      const int r = k - (c_hi_tot + sm.bc[1]);  // band keys still to keep, 1 <= r <= tot_band
+      if (r == tot_band) {  // the whole band is kept
+        for (int i = threadIdx.x; i < tot_band; i += kFThreads) {
+          const int s2 = bidx[i];
+          atomicOr(&bits[s2 >> 5], 1u << (s2 & 31));
+          atomicAdd(&chunk_cnt[s2 / kFChunk], 1);
+        }
+      } else {
+        // re-score the band four keys per warp call (the next four key rows
+        // are loaded while the current ones are scored)
+        const double w_lane = lane < HI ? static_cast<double>(w_pre) : 0.0;
+        uint32_t* my_kst = kst_all + warp * 512;
+        int b = 4 * warp;
+        uint2 raw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)], DI) : make_uint2(0u, 0u);
+        for (; b < tot_band; b += 4 * kFWarps) {
+          const int bn = b + 4 * kFWarps;
+          uint2 nraw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)], DI)
+                                    : make_uint2(0u, 0u);
+          const double xl = rescore4<DI>(qhi, w_lane, raw, my_kst, HI);
+          if (lane < 4 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, kWinCap, 52))
+            bx[b + lane] = d2key(xl);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
+        }
+        __syncthreads();
+        // rank by (X desc, key asc): a warp takes four band keys at a time
+        for (int b0 = 4 * warp; b0 < tot_band; b0 += 4 * kFWarps) {
+          unsigned long long xb[4];
+          int sb[4], rank[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int bb = min(b0 + e, tot_band - 1);
+            xb[e] = bx[bb];
+            sb[e] = bidx[bb];
+            rank[e] = 0;
+          }
+          for (int o = lane; o < tot_band; o += 32) {
+            const unsigned long long xo = bx[o];
+            const int so = bidx[o];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rank[e] += (xo > xb[e]) || (xo == xb[e] && so < sb[e]);
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) rank[e] = __reduce_add_sync(0xffffffffu, rank[e]);
+          const int my_rank = lane == 0 ? rank[0] : lane == 1 ? rank[1] : lane == 2 ? rank[2] : rank[3];
+          const int my_s = lane == 0 ? sb[0] : lane == 1 ? sb[1] : lane == 2 ? sb[2] : sb[3];
+          if (lane < 4 && b0 + lane < tot_band && my_rank < r && DSA_IN_BOUNDS(a.ws, my_s, n, 53)) {
+            atomicOr(&bits[my_s >> 5], 1u << (my_s & 31));
+            atomicAdd(&chunk_cnt[my_s / kFChunk], 1);
+          }
+        }
+      }
+    }
+  }
+  if (redo) {  // (block-uniform) handed to topk_kernel
+    if (threadIdx.x == 0) {
+      out[0] = kRedoMarker;
+      atomicAdd(&a.ws->topk_redo, 1u);
+    }
+    return;
+  }
+  __syncthreads();
+
+  // ---- 5. emit: chunk offsets, then each chunk's kept keys in order
+  {
+    const int c0 = 2 * threadIdx.x;
+    const int v0 = c0 < n_chunks ? chunk_cnt[c0] : 0;
+    const int v1 = c0 + 1 < n_chunks ? chunk_cnt[c0 + 1] : 0;
+    unsigned long long tot;
+    const int base = static_cast<int>(block_excl_scan64<kFThreads>(static_cast<unsigned long long>(v0 + v1), &tot, sm));
+    if (c0 < n_chunks) chunk_cnt[c0] = base;
+    if (c0 + 1 < n_chunks) chunk_cnt[c0 + 1] = base + v0;
+    if (threadIdx.x == 0 && static_cast<int>(tot) != k) report(a.ws, kDevInternal, static_cast<unsigned>(row));
+    // (2 * kFThreads chunks cover 49,152 keys)
+  }
+  __syncthreads();
+  int32_t* stage = hist;  // the selection, assembled in shared memory
+  for (int c = warp; c < n_chunks; c += kFWarps) {
+    const int s0 = c * kFChunk + 4 * lane;
+    float v[4];
+    if (s0 + 3 < n) {
+      const float4 f4 = __ldg(reinterpret_cast<const float4*>(srow + s0));
+      v[0] = f4.x; v[1] = f4.y; v[2] = f4.z; v[3] = f4.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = s0 + e < n ? __ldg(srow + s0 + e) : -INFINITY;
+    }
+    const uint32_t word = bits[min(s0, n - 1) >> 5];
+    bool keep[4];
+    int cnt = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int s = s0 + e;
+      keep[e] = s < n && (v[e] > whi_f || ((word >> (s & 31)) & 1u));
+      cnt += keep[e];
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = chunk_cnt[c] + incl - cnt;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (keep[e]) {
+        if (pos < k && DSA_IN_BOUNDS(a.ws, pos, kBins, 54)) stage[pos] = s0 + e;
+        ++pos;
+      }
+    }
+  }
+  __syncthreads();
+  if ((k & 3) == 0) {
+    for (int i = threadIdx.x; i < k / 4; i += kFThreads)
+      reinterpret_cast<int4*>(out)[i] = reinterpret_cast<const int4*>(stage)[i];
+  } else {
+    for (int i = threadIdx.x; i < k; i += kFThreads) out[i] = stage[i];
+  }
+}
+
 __global__ void key_norm_max_kernel(const uint16_t* __restrict__ k_idx, int T, int DI,
                                     WsHeader* ws) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -963,8 +1334,37 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   a.seg_len = 0;
   a.n_seg = 0;
   a.cand = nullptr;
+  a.fw_chunks = 0;
+  a.fw_words = 0;
+  a.only_marked = 0;
   const bool refine = q_idx != nullptr;
   const TwoLevel t = two_level(d);
+  if (t.n_seg == 0 && refine && (d.d_idx == 128 || d.d_idx == 32) && d.n_idx_heads <= 32) {
+    // the window select, then topk_kernel on the rows it hands back
+    const int row_cap = d.q_pos0 + d.n_q;
+    a.fw_chunks = ((row_cap + kFChunk - 1) / kFChunk + 3) & ~3;
+    a.fw_words = ((row_cap + 31) / 32 + 3) & ~3;
+    const size_t bytes = sizeof(int) * kBins + sizeof(uint32_t) * 512 * kFWarps + kQRowBytes +
+                         (sizeof(unsigned long long) + sizeof(int)) * kWinCap +
+                         sizeof(int) * (a.fw_chunks + a.fw_words) + (sizeof(int) + sizeof(float)) * kWinCap;
+    cudaError_t e = cudaMemsetAsync(&ws->topk_redo, 0, sizeof(ws->topk_redo), st);
+    if (e != cudaSuccess) return e;
+    if (d.d_idx == 128) {
+      e = cudaFuncSetAttribute(topk_window_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(bytes));
+      if (e != cudaSuccess) return e;
+      topk_window_kernel<128><<<d.n_q, kFThreads, bytes, st>>>(a);
+    } else {
+      e = cudaFuncSetAttribute(topk_window_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(bytes));
+      if (e != cudaSuccess) return e;
+      topk_window_kernel<32><<<d.n_q, kFThreads, bytes, st>>>(a);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    a.only_marked = 1;
+    return launch_pass(a, row_cap, d.n_q, refine, st);
+  }
   if (t.n_seg == 0) return launch_pass(a, d.q_pos0 + d.n_q, d.n_q, refine, st);
   if (!cand) return cudaErrorInvalidValue;
   a.seg_len = t.seg_len;
