@@ -501,6 +501,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     key_off = seg * a.seg_len;
     n = min(a.seg_len, a.q_pos0 + row + 1 - key_off);
     out = a.cand + (static_cast<int64_t>(row) * a.n_seg + seg) * k;
+    if (a.only_marked) {  // redo only the segments the window select handed back
+      if (*reinterpret_cast<volatile unsigned int*>(&a.ws->topk_redo) == 0u) return;
+      if (*reinterpret_cast<volatile int32_t*>(out) != kRedoMarker) return;
+    }
     if (n <= 0) {  // a segment past the query's position
       for (int c = threadIdx.x; c < k; c += kThreads) out[c] = -1;
       return;
@@ -860,17 +864,34 @@ constexpr int kFWarps = kFThreads / 32;
 constexpr int kFChunk = 128;
 constexpr int kWinCap = 256;
 
-template <int DI>
+// kSeg: pass 1 of the long-row select (topk_kernel's pass 1): CTA (row,
+// segment) selects among the segment's keys key_off .. key_off + n - 1 and
+// writes them to the candidate buffer.
+template <int DI, bool kSeg>
 __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ Scratch sm;
   __shared__ int s_ncand, s_chi;
   const int k = a.k;
-  const int row = blockIdx.x;
-  const int n = a.q_pos0 + row + 1;
-  int32_t* out = a.idx + static_cast<int64_t>(row) * k;
-  if (n <= k) {  // every causal key is kept
-    for (int c = threadIdx.x; c < k; c += kFThreads) out[c] = c < n ? c : -1;
+  int row, n, key_off = 0;
+  int32_t* out;
+  if (kSeg) {
+    row = blockIdx.x / a.n_seg;
+    const int seg = blockIdx.x - row * a.n_seg;
+    key_off = seg * a.seg_len;
+    n = min(a.seg_len, a.q_pos0 + row + 1 - key_off);
+    out = a.cand + (static_cast<int64_t>(row) * a.n_seg + seg) * k;
+    if (n <= 0) {  // a segment past the query's position
+      for (int c = threadIdx.x; c < k; c += kFThreads) out[c] = -1;
+      return;
+    }
+  } else {
+    row = blockIdx.x;
+    n = a.q_pos0 + row + 1;
+    out = a.idx + static_cast<int64_t>(row) * k;
+  }
+  if (n <= k) {  // every key is kept
+    for (int c = threadIdx.x; c < k; c += kFThreads) out[c] = c < n ? c + key_off : -1;
     return;
   }
   const int HI = a.HI;
@@ -943,7 +964,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   }
 
   // ---- 1. the row's range
-  const float* srow = a.scores + static_cast<int64_t>(row) * a.ld;
+  const float* srow = a.scores + static_cast<int64_t>(row) * a.ld + key_off;  // (key_off % 4 == 0)
   const float4* s4 = reinterpret_cast<const float4*>(srow);
   const int n4 = n >> 2;
   float mn = INFINITY, mx = -INFINITY;
@@ -1079,13 +1100,14 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
         uint2 raw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)], DI) : make_uint2(0u, 0u);
+          raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)] + key_off, DI)
+                                : make_uint2(0u, 0u);
         for (; b < tot_band; b += 4 * kFWarps) {
           const int bn = b + 4 * kFWarps;
           uint2 nraw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)], DI)
+            nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)] + key_off, DI)
                                     : make_uint2(0u, 0u);
           const double xl = rescore4<DI>(qhi, w_lane, raw, my_kst, HI);
           if (lane < 4 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, kWinCap, 52))
@@ -1175,7 +1197,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (keep[e]) {
-        if (pos < k && DSA_IN_BOUNDS(a.ws, pos, kBins, 54)) stage[pos] = s0 + e;
+        if (pos < k && DSA_IN_BOUNDS(a.ws, pos, kBins, 54)) stage[pos] = s0 + e + key_off;
         ++pos;
       }
     }
@@ -1307,6 +1329,27 @@ cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStre
   return launch_kernel(a, grid, bytes, refine, st);
 }
 
+// The window select over `grid` rows (or row segments, seg) of at most
+// row_cap keys, after clearing the count of handed-back rows.
+cudaError_t launch_window(TopkArgs& a, int row_cap, int grid, bool seg, cudaStream_t st) {
+  a.fw_chunks = ((row_cap + kFChunk - 1) / kFChunk + 3) & ~3;
+  a.fw_words = ((row_cap + 31) / 32 + 3) & ~3;
+  const size_t bytes = sizeof(int) * kBins + sizeof(uint32_t) * 512 * kFWarps + kQRowBytes +
+                       (sizeof(unsigned long long) + sizeof(int)) * kWinCap +
+                       sizeof(int) * (a.fw_chunks + a.fw_words) + (sizeof(int) + sizeof(float)) * kWinCap;
+  cudaError_t e = cudaMemsetAsync(&a.ws->topk_redo, 0, sizeof(a.ws->topk_redo), st);
+  if (e != cudaSuccess) return e;
+  auto go = [&](auto kernel) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(bytes));
+    if (e2 != cudaSuccess) return e2;
+    kernel<<<grid, kFThreads, bytes, st>>>(a);
+    return cudaGetLastError();
+  };
+  if (a.DI == 128) return seg ? go(topk_window_kernel<128, true>) : go(topk_window_kernel<128, false>);
+  return seg ? go(topk_window_kernel<32, true>) : go(topk_window_kernel<32, false>);
+}
+
 }  // namespace
 
 size_t topk_cand_bytes(const dsa_dims& d) {
@@ -1339,28 +1382,11 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   a.only_marked = 0;
   const bool refine = q_idx != nullptr;
   const TwoLevel t = two_level(d);
-  if (t.n_seg == 0 && refine && (d.d_idx == 128 || d.d_idx == 32) && d.n_idx_heads <= 32) {
+  const bool window = refine && (d.d_idx == 128 || d.d_idx == 32) && d.n_idx_heads <= 32;
+  if (t.n_seg == 0 && window) {
     // the window select, then topk_kernel on the rows it hands back
     const int row_cap = d.q_pos0 + d.n_q;
-    a.fw_chunks = ((row_cap + kFChunk - 1) / kFChunk + 3) & ~3;
-    a.fw_words = ((row_cap + 31) / 32 + 3) & ~3;
-    const size_t bytes = sizeof(int) * kBins + sizeof(uint32_t) * 512 * kFWarps + kQRowBytes +
-                         (sizeof(unsigned long long) + sizeof(int)) * kWinCap +
-                         sizeof(int) * (a.fw_chunks + a.fw_words) + (sizeof(int) + sizeof(float)) * kWinCap;
-    cudaError_t e = cudaMemsetAsync(&ws->topk_redo, 0, sizeof(ws->topk_redo), st);
-    if (e != cudaSuccess) return e;
-    if (d.d_idx == 128) {
-      e = cudaFuncSetAttribute(topk_window_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(bytes));
-      if (e != cudaSuccess) return e;
-      topk_window_kernel<128><<<d.n_q, kFThreads, bytes, st>>>(a);
-    } else {
-      e = cudaFuncSetAttribute(topk_window_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(bytes));
-      if (e != cudaSuccess) return e;
-      topk_window_kernel<32><<<d.n_q, kFThreads, bytes, st>>>(a);
-    }
-    e = cudaGetLastError();
+    cudaError_t e = launch_window(a, row_cap, d.n_q, false, st);
     if (e != cudaSuccess) return e;
     a.only_marked = 1;
     return launch_pass(a, row_cap, d.n_q, refine, st);
@@ -1371,8 +1397,15 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   a.n_seg = t.n_seg;
   a.cand = static_cast<int32_t*>(cand);
   a.pass = 1;
-  cudaError_t e = launch_pass(a, t.seg_len, d.n_q * t.n_seg, refine, st);
+  cudaError_t e;
+  if (window) {  // the segments through the window select, handed-back ones through topk_kernel
+    e = launch_window(a, t.seg_len, d.n_q * t.n_seg, true, st);
+    if (e != cudaSuccess) return e;
+    a.only_marked = 1;
+  }
+  e = launch_pass(a, t.seg_len, d.n_q * t.n_seg, refine, st);
   if (e != cudaSuccess) return e;
+  a.only_marked = 0;
   a.pass = 2;
   return launch_pass(a, t.n_seg * d.top_k, d.n_q, refine, st);
 }
