@@ -453,6 +453,72 @@ __device__ __forceinline__ double rescore4(const uint32_t* __restrict__ qhi, dou
   return sum;
 }
 
+// rescore4 with the keys staged as full float64 values (8 bytes per dim)
+// instead of high words: the head dots then load their key operands as
+// ready float64 registers, with no moves to form register pairs. The same
+// operation order as rescore4. kst holds 4 x DI doubles, afterwards the
+// [4][34] products of the head sum.
+template <int DI>
+__device__ __forceinline__ double rescore4d(const uint32_t* __restrict__ qhi, double w_lane,
+                                            const uint2 (&raw)[4], double* __restrict__ kst, int HI) {
+  const int lane = threadIdx.x & 31;
+  if (lane * 4 < DI) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t w[2] = {raw[e].x, raw[e].y};
+      double2* dst = reinterpret_cast<double2*>(kst + e * DI + lane * 4);
+      dst[0] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[0] & 0xFFFFu)),
+                            bf16_to_f64(static_cast<uint16_t>(w[0] >> 16)));
+      dst[1] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[1] & 0xFFFFu)),
+                            bf16_to_f64(static_cast<uint16_t>(w[1] >> 16)));
+    }
+  }
+  __syncwarp();
+  double pr[4] = {0.0, 0.0, 0.0, 0.0};
+  if (lane < HI) {
+    const uint4* q4 = reinterpret_cast<const uint4*>(qhi + lane * (DI + 4));
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+    for (int c4 = 0; c4 < DI / 4; ++c4) {
+      const uint4 qq = q4[c4];
+      const double qd[4] = {__hiloint2double(static_cast<int>(qq.x), 0), __hiloint2double(static_cast<int>(qq.y), 0),
+                            __hiloint2double(static_cast<int>(qq.z), 0), __hiloint2double(static_cast<int>(qq.w), 0)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const double2* kp = reinterpret_cast<const double2*>(kst + e * DI + c4 * 4);
+        const double2 k01 = kp[0], k23 = kp[1];
+        acc[e] = fma(qd[0], k01.x, acc[e]);
+        acc[e] = fma(qd[1], k01.y, acc[e]);
+        acc[e] = fma(qd[2], k23.x, acc[e]);
+        acc[e] = fma(qd[3], k23.y, acc[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pr[e] = __dmul_rn(w_lane, acc[e] > 0.0 ? acc[e] : 0.0);
+  }
+  __syncwarp();
+  double* prod = kst;
+  if (lane < HI) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) prod[e * 34 + lane] = pr[e];
+  }
+  __syncwarp();
+  double sum = 0.0;
+  if (lane < 4) {
+    const double2* pe = reinterpret_cast<const double2*>(prod + lane * 34);
+#pragma unroll
+    for (int j2 = 0; j2 < 16; ++j2) {
+      if (2 * j2 < HI) {
+        const double2 v = pe[j2];
+        sum = __dadd_rn(sum, v.x);
+        sum = __dadd_rn(sum, v.y);  // HI is even
+      }
+    }
+  }
+  __syncwarp();
+  return sum;
+}
+
 struct TopkArgs {
   const float* scores;
   int64_t ld;
@@ -863,6 +929,8 @@ constexpr int kFThreads = 192;
 constexpr int kFWarps = kFThreads / 32;
 constexpr int kFChunk = 128;
 constexpr int kWinCap = 256;
+// hist (2,048 ints), or the re-score's key staging: 4 keys x 128 float64 per warp
+constexpr int kFRegionBytes = (kBins * 4 > kFWarps * 4 * 128 * 8) ? kBins * 4 : kFWarps * 4 * 128 * 8;
 
 // kSeg: pass 1 of the long-row select (topk_kernel's pass 1): CTA (row,
 // segment) selects among the segment's keys key_off .. key_off + n - 1 and
@@ -901,8 +969,9 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   // re-score | q row (float64 high words) | band cache | chunk counts |
   // kept-key bitmap | window keys and scores
   int* hist = reinterpret_cast<int*>(smem);
-  uint32_t* kst_all = reinterpret_cast<uint32_t*>(smem + kBins * 4);
-  uint32_t* qhi = kst_all + kFWarps * 512;
+  // (the re-score's float64 key staging overlays hist, idle in that phase)
+  double* kst_all = reinterpret_cast<double*>(smem);
+  uint32_t* qhi = reinterpret_cast<uint32_t*>(smem + kFRegionBytes);
   unsigned long long* bx = reinterpret_cast<unsigned long long*>(
       reinterpret_cast<unsigned char*>(qhi) + kQRowBytes);
   int* bidx = reinterpret_cast<int*>(bx + kWinCap);
@@ -1095,7 +1164,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
         // re-score the band four keys per warp call (the next four key rows
         // are loaded while the current ones are scored)
         const double w_lane = lane < HI ? static_cast<double>(w_pre) : 0.0;
-        uint32_t* my_kst = kst_all + warp * 512;
+        double* my_kst = kst_all + warp * 4 * DI;
         int b = 4 * warp;
         uint2 raw[4];
 #pragma unroll
@@ -1109,7 +1178,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
           for (int e = 0; e < 4; ++e)
             nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)] + key_off, DI)
                                     : make_uint2(0u, 0u);
-          const double xl = rescore4<DI>(qhi, w_lane, raw, my_kst, HI);
+          const double xl = rescore4d<DI>(qhi, w_lane, raw, my_kst, HI);
           if (lane < 4 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, kWinCap, 52))
             bx[b + lane] = d2key(xl);
 #pragma unroll
@@ -1334,7 +1403,7 @@ cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStre
 cudaError_t launch_window(TopkArgs& a, int row_cap, int grid, bool seg, cudaStream_t st) {
   a.fw_chunks = ((row_cap + kFChunk - 1) / kFChunk + 3) & ~3;
   a.fw_words = ((row_cap + 31) / 32 + 3) & ~3;
-  const size_t bytes = sizeof(int) * kBins + sizeof(uint32_t) * 512 * kFWarps + kQRowBytes +
+  const size_t bytes = kFRegionBytes + kQRowBytes +
                        (sizeof(unsigned long long) + sizeof(int)) * kWinCap +
                        sizeof(int) * (a.fw_chunks + a.fw_words) + (sizeof(int) + sizeof(float)) * kWinCap;
   cudaError_t e = cudaMemsetAsync(&a.ws->topk_redo, 0, sizeof(a.ws->topk_redo), st);
