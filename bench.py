@@ -53,11 +53,17 @@ PROFILED_DRAM_BYTES_PER_LAUNCH: dict = {
     ("sparse_attn_tc", "chunk8k_ctx17k"): 389_857_536 + 242_595_840,
 }
 # the CUDA kernel behind each timed entry point (the layer's own launch configuration)
-KERNEL_OF = {"index_scores": "index_scores_tc", "topk_select": "topk_kernel",
+KERNEL_OF = {"index_scores": "index_scores_tc", "topk_select": "topk_window_kernel",
              "sparse_attn": "sparse_attn_tc"}
 
-KERNELS_PER_LAYER = 5  # indexer scores, indexer key-norm max, top-k, attention key-norm max, attention
-# (the FP8 indexer variant adds the e4m3 forms of the keys and of the queries)
+def kernels_per_layer(d) -> int:
+    """Kernels one layer call launches: the two key-norm passes, the indexer,
+    the top-k's window select and its redo pass over handed-back rows (whose
+    CTAs exit at once when there are none), a second top-k pass for rows past
+    49,152 keys, and the attention; the FP8 indexer adds the e4m3 forms of the
+    keys and of the queries."""
+    two_pass = d.q_pos0 + d.n_q > 49152
+    return 6 + (1 if two_pass else 0) + (2 if d.flags & 1 else 0)
 E2E_SUB_CHUNKS = (2, 4, 8, 16, 64)  # query sub-chunk counts tried for the host-buffer call (copies overlap the layer)
 
 
@@ -559,7 +565,7 @@ def run_ours(args):
                 "h2d_alone_ms": h2d_only_ms, "d2h_alone_ms": d2h_only_ms,
                 "h2d_and_d2h_together_ms": both_ms,
                 "warmup_ms_by_sub_chunks": {str(k): round(v, 3) for k, v in tried.items()}},
-        "gpu_launches": (KERNELS_PER_LAYER + (2 if args.fp8_indexer else 0)) * args.steps,
+        "gpu_launches": kernels_per_layer(d) * args.steps,
         "roofline": roof,
         "clocks": clocks.summary(),
     }
@@ -681,7 +687,7 @@ def run_split(args):
         "tflops": tflops, "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
         "e2e": {"value": d.n_q / (e2e_ms / 1e3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": KERNELS_PER_LAYER * args.steps,
+        "gpu_launches": kernels_per_layer(d) * args.steps,
         "clocks": clocks.summary(),
     }
     if world > 1:

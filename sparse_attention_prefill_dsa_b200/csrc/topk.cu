@@ -554,42 +554,32 @@ struct TopkArgs {
 // select (a template parameter, so that the one-level kernel carries none of
 // the other passes' key mapping)
 template <bool kRefine, int kPass>
-__global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ Scratch sm;
+__device__ __forceinline__ void topk_row(const TopkArgs& a, int blk, unsigned char* smem, Scratch& sm) {
   const int k = a.k;
   int row, n, key_off = 0;
   const int32_t* kmap = nullptr;  // pass 2: key of each position of the candidate row
   int32_t* out;
   if (kPass == 1) {  // segment seg of the row
-    row = blockIdx.x / a.n_seg;
-    const int seg = blockIdx.x - row * a.n_seg;
+    row = blk / a.n_seg;
+    const int seg = blk - row * a.n_seg;
     key_off = seg * a.seg_len;
     n = min(a.seg_len, a.q_pos0 + row + 1 - key_off);
     out = a.cand + (static_cast<int64_t>(row) * a.n_seg + seg) * k;
-    if (a.only_marked) {  // redo only the segments the window select handed back
-      if (*reinterpret_cast<volatile unsigned int*>(&a.ws->topk_redo) == 0u) return;
-      if (*reinterpret_cast<volatile int32_t*>(out) != kRedoMarker) return;
-    }
     if (n <= 0) {  // a segment past the query's position
       for (int c = threadIdx.x; c < k; c += kThreads) out[c] = -1;
       return;
     }
   } else if (kPass == 2) {  // the row's candidates
-    row = blockIdx.x;
+    row = blk;
     const int t = a.q_pos0 + row;
     const int nv = t / a.seg_len + 1;  // non-empty segments
     n = (nv - 1) * k + min(k, t + 1 - (nv - 1) * a.seg_len);
     kmap = a.cand + static_cast<int64_t>(row) * a.n_seg * k;
     out = a.idx + static_cast<int64_t>(row) * k;
   } else {
-    row = blockIdx.x;
+    row = blk;
     n = a.q_pos0 + row + 1;
     out = a.idx + static_cast<int64_t>(row) * k;
-    if (a.only_marked) {  // redo only the rows the window select handed back
-      if (*reinterpret_cast<volatile unsigned int*>(&a.ws->topk_redo) == 0u) return;
-      if (*reinterpret_cast<volatile int32_t*>(out) != kRedoMarker) return;
-    }
   }
 
   if (n <= k) {  // every key of the row (or segment, or candidate list) is kept
@@ -899,6 +889,42 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
         return v > hi_f ? kAbove : kBelow;
       },
       sm, a.ws, row, -1, key_off, kmap);
+}
+
+
+// One CTA per row (or row segment, or candidate list); with only_marked a
+// grid of a few CTAs per SM scans for the rows (pass 0) or row segments
+// (pass 1) the window select handed back and redoes those alone.
+template <bool kRefine, int kPass>
+__global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ Scratch sm;
+  if (!a.only_marked) {
+    topk_row<kRefine, kPass>(a, blockIdx.x, smem, sm);
+    return;
+  }
+  if (*reinterpret_cast<volatile unsigned int*>(&a.ws->topk_redo) == 0u) return;
+  __shared__ unsigned int s_mask[kWarps];  // per warp: which of its 32 rows are marked
+  const int n_blk = kPass == 1 ? a.n_q * a.n_seg : a.n_q;
+  int32_t* const base_out = kPass == 1 ? a.cand : a.idx;
+  for (int base = blockIdx.x * kThreads; base < n_blk; base += gridDim.x * kThreads) {
+    const int b = base + static_cast<int>(threadIdx.x);
+    const bool marked =
+        b < n_blk &&
+        *reinterpret_cast<volatile int32_t*>(base_out + static_cast<int64_t>(b) * a.k) == kRedoMarker;
+    const unsigned int m = __ballot_sync(0xffffffffu, marked);
+    if ((threadIdx.x & 31) == 0) s_mask[threadIdx.x >> 5] = m;
+    __syncthreads();
+    for (int w = 0; w < kWarps; ++w) {
+      unsigned int mw = s_mask[w];
+      while (mw) {
+        const int bit = __ffs(mw) - 1;
+        mw &= mw - 1u;
+        topk_row<kRefine, kPass>(a, base + 32 * w + bit, smem, sm);
+        __syncthreads();
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1352,6 +1378,13 @@ cudaError_t launch_kernel(const TopkArgs& a, int grid, size_t bytes, bool refine
   }
 }
 
+int num_sms_topk() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 // One launch of topk_kernel over `grid` CTAs with rows of up to `row_cap`
 // staged scores: picks the shared-memory layout (two CTAs per SM with eight
 // re-scoring warps, else one with eight, else one with four) and launches.
@@ -1360,7 +1393,8 @@ cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStre
   int max_smem = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const size_t static_bytes = sizeof(Scratch) + 64;
+  // static shared memory of topk_kernel: Scratch and the redo scan's row masks
+  const size_t static_bytes = sizeof(Scratch) + sizeof(unsigned int) * kWarps + 64;
   size_t bytes = sizeof(float) * a.n_cap + sizeof(int) * kBins + sizeof(float) * kCandCap;
   a.bcap = 0;
   a.kst_extra = 0;
@@ -1394,6 +1428,10 @@ cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStre
     }
   } else if (static_cast<size_t>(max_smem) < bytes + static_bytes) {
     return cudaErrorInvalidConfiguration;
+  }
+  if (a.only_marked) {  // the redo pass scans for handed-back rows with a few CTAs per SM
+    const int scan_grid = 2 * num_sms_topk();
+    if (grid > scan_grid) grid = scan_grid;
   }
   return launch_kernel(a, grid, bytes, refine, st);
 }
