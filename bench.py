@@ -48,9 +48,9 @@ L2_FLUSH_BYTES = 256 << 20
 # its kernel changes after the capture.
 # key: (CUDA kernel, workload); value: bytes per launch
 PROFILED_DRAM_BYTES_PER_LAUNCH: dict = {
-    ("index_scores_tc", "chunk8k_ctx17k"): 256_241_408 + 394_494_464,
-    ("topk_kernel", "chunk8k_ctx17k"): 514_805_760 + 57_556_736,
-    ("sparse_attn_tc", "chunk8k_ctx17k"): 389_857_536 + 242_595_840,
+    ("index_scores_tc", "chunk8k_ctx17k"): 255_553_536 + 394_548_992,
+    ("topk_window_kernel", "chunk8k_ctx17k"): 517_252_608 + 57_187_328,
+    ("sparse_attn_tc", "chunk8k_ctx17k"): 389_560_064 + 243_148_800,
 }
 # the CUDA kernel behind each timed entry point (the layer's own launch configuration)
 KERNEL_OF = {"index_scores": "index_scores_tc", "topk_select": "topk_window_kernel",
