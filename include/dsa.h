@@ -56,7 +56,7 @@ typedef struct dsa_dims {
   int32_t d_idx;       /* indexer head width D_I                                      */
   int32_t top_k;       /* keys kept per query, 1..DSA_MAX_TOPK                        */
   float softmax_scale; /* multiplies the attention logits                             */
-  uint32_t flags;      /* 0, or DSA_FLAG_FP8_INDEXER in the whole-layer calls         */
+  uint32_t flags;      /* 0, or the DSA_FLAG_* options below where a call accepts them */
 } dsa_dims;
 
 /* dims.flags: the whole-layer calls (dsa_prefill_layer, dsa_decode_layer,

@@ -6,6 +6,13 @@
 // reading this library fixes, in the spirit of the TensorFold issue #743
 // thread, whose maintainers grant no tie exception between chunkings.
 //
+// Two kernels. With the indexer inputs given (the exact mode of every layer
+// call) topk_window_kernel, the window select described further down, runs
+// first: a 192-thread CTA per row that keeps only a window of the row around
+// its k-th value, four rows per SM. Rows it hands back (heavy ties, a
+// degenerate range), and the float32-only mode, run topk_kernel, the bucket
+// select described here:
+//
 // One CTA (384 threads) per query row; the row's float32 scores s = 0..t are
 // staged once in shared memory (t + 1 <= 49152 -> at most 192 KB). Longer
 // rows take two levels: pass 1 selects the top-k of every segment of at most
