@@ -550,10 +550,10 @@ struct TopkArgs {
   // pass 0 is the one-level select.
   int pass, seg_len, n_seg;
   int32_t* cand;
-  // the window select (topk_window_kernel): shared-memory sizes of its chunk
-  // counts and kept-key bitmap; only_marked makes topk_kernel redo only the
-  // rows the window select handed back
-  int fw_chunks, fw_words;
+  // the window select (topk_window_kernel): words of its kept-key bitmap;
+  // only_marked makes topk_kernel redo only the rows the window select
+  // handed back
+  int fw_words;
   int only_marked;
 };
 
@@ -943,17 +943,17 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 //   1. the row's range [L, U];
 //   2. a histogram over 2,048 buckets of the range, and the bucket b* that
 //      holds the k-th largest float score v;
-//   3. the window pass: per chunk the number of keys above a window around
-//      b* widened by 2 delta on either side (delta as in topk_kernel), and
-//      the window's keys collected with their scores. Every key within
-//      2 delta of v is in the window, so v, the keys certainly kept
-//      (above v + 2 delta) and the band [v - 2 delta, v + 2 delta] follow from
-//      the window alone;
+//   3. the window pass: the keys above a window around b*, widened by
+//      2 delta on either side (delta as in topk_kernel), go into a bitmap of
+//      the row, and the window's keys are collected with their scores. Every
+//      key within 2 delta of v is in the window, so v, the keys certainly
+//      kept (above v + 2 delta) and the band [v - 2 delta, v + 2 delta] follow
+//      from the window alone;
 //   4. the band re-scored in float64 in the contract's order and ranked by
 //      (X desc, key asc), exactly as in topk_kernel; the window's kept keys
-//      are marked in a bitmap and counted in their chunks;
-//   5. the emit: a scan of the chunk counts places each chunk's kept keys
-//      (the keys above the window and the marked ones) in ascending order.
+//      are added to the bitmap;
+//   5. the emit: a scan of the bitmap words' populations places the kept
+//      keys in ascending order.
 // A row whose range is a single value or too wide for a float bucket scale,
 // or whose window holds more than kWinCap keys (heavy ties), is handed back:
 // its first index is set to kRedoMarker and counted in the workspace header,
@@ -998,8 +998,8 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   const int HI = a.HI;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_chunks = (n + kFChunk - 1) / kFChunk;
-  // shared memory: hist (later the emit's staging) | key staging of the
-  // re-score | q row (float64 high words) | band cache | chunk counts |
+  // shared memory: hist (later the emit's staging; the re-score's key
+  // staging in between) | q row (float64 high words) | band cache |
   // kept-key bitmap | window keys and scores
   int* hist = reinterpret_cast<int*>(smem);
   // (the re-score's float64 key staging overlays hist, idle in that phase)
@@ -1008,8 +1008,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   unsigned long long* bx = reinterpret_cast<unsigned long long*>(
       reinterpret_cast<unsigned char*>(qhi) + kQRowBytes);
   int* bidx = reinterpret_cast<int*>(bx + kWinCap);
-  int* chunk_cnt = bidx + kWinCap;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(chunk_cnt + a.fw_chunks);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(bidx + kWinCap);
   int* cand_pos = reinterpret_cast<int*>(bits + a.fw_words);
   float* cand_val = reinterpret_cast<float*>(cand_pos + kWinCap);
   const int qstride = DI + 4;
@@ -1017,8 +1016,6 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   const float w_pre = lane < HI ? __ldg(a.w_idx + static_cast<int64_t>(row) * HI + lane) : 0.f;
   const unsigned long long kmax_bits = *reinterpret_cast<volatile unsigned long long*>(&a.ws->kmax_bits);
   for (int b = threadIdx.x; b < kBins; b += kFThreads) hist[b] = 0;
-  for (int c = threadIdx.x; c < n_chunks; c += kFThreads) chunk_cnt[c] = 0;
-  for (int w = threadIdx.x; w < (n + 31) / 32; w += kFThreads) bits[w] = 0u;
   if (threadIdx.x == 0) {
     s_ncand = 0;
     s_chi = 0;
@@ -1123,10 +1120,13 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
         for (int e = 0; e < 4; ++e) v[e] = s0 + e < n ? __ldg(srow + s0 + e) : -INFINITY;
       }
       int above = 0;
+      uint32_t mine = 0u;  // this lane's keys above the window, as bits of its chunk word
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float f = v[e];
-        above += f > whi_f;
+        const bool up = f > whi_f;
+        above += up;
+        mine |= static_cast<uint32_t>(up) << (4 * (lane & 7) + e);
         if (s0 + e < n && f >= wlo_f && f <= whi_f) {
           const int pos = atomicAdd(&s_ncand, 1);
           if (pos < kWinCap) {
@@ -1135,9 +1135,15 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
           }
         }
       }
-      above = __reduce_add_sync(0xffffffffu, above);
-      if (lane == 0 && DSA_IN_BOUNDS(a.ws, c, a.fw_chunks, 51)) chunk_cnt[c] = above;
-      c_hi += above;
+      // the chunk's four bitmap words (keys c * 128 + 32 g .. + 31 from lanes
+      // 8 g .. 8 g + 7), written by one lane each; the window's kept keys are
+      // added after this pass
+      mine |= __shfl_xor_sync(0xffffffffu, mine, 1);
+      mine |= __shfl_xor_sync(0xffffffffu, mine, 2);
+      mine |= __shfl_xor_sync(0xffffffffu, mine, 4);
+      if ((lane & 7) == 0 && DSA_IN_BOUNDS(a.ws, c * 4 + (lane >> 3), a.fw_words, 51))
+        bits[c * 4 + (lane >> 3)] = mine;
+      c_hi += __reduce_add_sync(0xffffffffu, above);
     }
     if (lane == 0) atomicAdd(&s_chi, c_hi);
     __syncthreads();
@@ -1173,10 +1179,7 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
           const unsigned mb = __ballot_sync(0xffffffffu, in_band);
           nin += __popc(__ballot_sync(0xffffffffu, above2));
           if (in_band) bidx[nb + __popc(mb & ((1u << lane) - 1u))] = s2;
-          if (above2) {
-            atomicOr(&bits[s2 >> 5], 1u << (s2 & 31));
-            atomicAdd(&chunk_cnt[s2 / kFChunk], 1);
-          }
+          if (above2) atomicOr(&bits[s2 >> 5], 1u << (s2 & 31));
           nb += __popc(mb);
         }
         if (lane == 0) {
@@ -1191,7 +1194,6 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
         for (int i = threadIdx.x; i < tot_band; i += kFThreads) {
           const int s2 = bidx[i];
           atomicOr(&bits[s2 >> 5], 1u << (s2 & 31));
-          atomicAdd(&chunk_cnt[s2 / kFChunk], 1);
         }
       } else {
         // re-score the band four keys per warp call (the next four key rows
@@ -1241,7 +1243,6 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
           const int my_s = lane == 0 ? sb[0] : lane == 1 ? sb[1] : lane == 2 ? sb[2] : sb[3];
           if (lane < 4 && b0 + lane < tot_band && my_rank < r && DSA_IN_BOUNDS(a.ws, my_s, n, 53)) {
             atomicOr(&bits[my_s >> 5], 1u << (my_s & 31));
-            atomicAdd(&chunk_cnt[my_s / kFChunk], 1);
           }
         }
       }
@@ -1256,50 +1257,24 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
   }
   __syncthreads();
 
-  // ---- 5. emit: chunk offsets, then each chunk's kept keys in order
-  {
-    const int c0 = 2 * threadIdx.x;
-    const int v0 = c0 < n_chunks ? chunk_cnt[c0] : 0;
-    const int v1 = c0 + 1 < n_chunks ? chunk_cnt[c0 + 1] : 0;
-    unsigned long long tot;
-    const int base = static_cast<int>(block_excl_scan64<kFThreads>(static_cast<unsigned long long>(v0 + v1), &tot, sm));
-    if (c0 < n_chunks) chunk_cnt[c0] = base;
-    if (c0 + 1 < n_chunks) chunk_cnt[c0 + 1] = base + v0;
-    if (threadIdx.x == 0 && static_cast<int>(tot) != k) report(a.ws, kDevInternal, static_cast<unsigned>(row));
-    // (2 * kFThreads chunks cover 49,152 keys)
-  }
-  __syncthreads();
+  // ---- 5. emit: the bitmap holds exactly the kept keys; a scan of the words'
+  // populations places each thread's words (a contiguous run) in order
   int32_t* stage = hist;  // the selection, assembled in shared memory
-  for (int c = warp; c < n_chunks; c += kFWarps) {
-    const int s0 = c * kFChunk + 4 * lane;
-    float v[4];
-    if (s0 + 3 < n) {
-      const float4 f4 = __ldg(reinterpret_cast<const float4*>(srow + s0));
-      v[0] = f4.x; v[1] = f4.y; v[2] = f4.z; v[3] = f4.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = s0 + e < n ? __ldg(srow + s0 + e) : -INFINITY;
-    }
-    const uint32_t word = bits[min(s0, n - 1) >> 5];
-    bool keep[4];
+  {
+    const int n_words = (n + 31) / 32;
+    const int per = (n_words + kFThreads - 1) / kFThreads;
+    const int w0 = min(static_cast<int>(threadIdx.x) * per, n_words), w1 = min(w0 + per, n_words);
     int cnt = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int s = s0 + e;
-      keep[e] = s < n && (v[e] > whi_f || ((word >> (s & 31)) & 1u));
-      cnt += keep[e];
-    }
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = chunk_cnt[c] + incl - cnt;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (keep[e]) {
-        if (pos < k && DSA_IN_BOUNDS(a.ws, pos, kBins, 54)) stage[pos] = s0 + e + key_off;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+    unsigned long long tot;
+    int pos = static_cast<int>(block_excl_scan64<kFThreads>(static_cast<unsigned long long>(cnt), &tot, sm));
+    if (threadIdx.x == 0 && static_cast<int>(tot) != k) report(a.ws, kDevInternal, static_cast<unsigned>(row));
+    for (int w = w0; w < w1; ++w) {
+      uint32_t m = bits[w];
+      while (m) {
+        const int bit = __ffs(m) - 1;
+        m &= m - 1u;
+        if (pos < k && DSA_IN_BOUNDS(a.ws, pos, kBins, 54)) stage[pos] = 32 * w + bit + key_off;
         ++pos;
       }
     }
@@ -1446,11 +1421,10 @@ cudaError_t launch_pass(TopkArgs a, int row_cap, int grid, bool refine, cudaStre
 // The window select over `grid` rows (or row segments, seg) of at most
 // row_cap keys, after clearing the count of handed-back rows.
 cudaError_t launch_window(TopkArgs& a, int row_cap, int grid, bool seg, cudaStream_t st) {
-  a.fw_chunks = ((row_cap + kFChunk - 1) / kFChunk + 3) & ~3;
   a.fw_words = ((row_cap + 31) / 32 + 3) & ~3;
   const size_t bytes = kFRegionBytes + kQRowBytes +
                        (sizeof(unsigned long long) + sizeof(int)) * kWinCap +
-                       sizeof(int) * (a.fw_chunks + a.fw_words) + (sizeof(int) + sizeof(float)) * kWinCap;
+                       sizeof(int) * a.fw_words + (sizeof(int) + sizeof(float)) * kWinCap;
   cudaError_t e = cudaMemsetAsync(&a.ws->topk_redo, 0, sizeof(a.ws->topk_redo), st);
   if (e != cudaSuccess) return e;
   auto go = [&](auto kernel) -> cudaError_t {
@@ -1491,7 +1465,6 @@ cudaError_t launch_topk(const dsa_dims& d, const float* scores, int64_t ld, cons
   a.seg_len = 0;
   a.n_seg = 0;
   a.cand = nullptr;
-  a.fw_chunks = 0;
   a.fw_words = 0;
   a.only_marked = 0;
   const bool refine = q_idx != nullptr;
