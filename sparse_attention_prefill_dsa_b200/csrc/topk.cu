@@ -460,58 +460,62 @@ __device__ __forceinline__ double rescore4(const uint32_t* __restrict__ qhi, dou
   return sum;
 }
 
-// rescore4 with the keys staged as full float64 values (8 bytes per dim)
-// instead of high words: the head dots then load their key operands as
-// ready float64 registers, with no moves to form register pairs. The same
-// operation order as rescore4. kst holds 4 x DI doubles, afterwards the
-// [4][34] products of the head sum.
+// rescore4 for eight keys per call (eight independent float64 chains per
+// lane instead of four), the keys staged as float64 high words (8 x DI
+// words). The same operation order as rescore4. Lane e < 8 returns key e's
+// score; kst afterwards holds the [8][34] products of the head sum.
 template <int DI>
-__device__ __forceinline__ double rescore4d(const uint32_t* __restrict__ qhi, double w_lane,
-                                            const uint2 (&raw)[4], double* __restrict__ kst, int HI) {
+__device__ __forceinline__ double rescore8h(const uint32_t* __restrict__ qhi, double w_lane,
+                                            const uint2 (&raw)[8], uint32_t* __restrict__ kst, int HI) {
   const int lane = threadIdx.x & 31;
   if (lane * 4 < DI) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 8; ++e) {
       const uint32_t w[2] = {raw[e].x, raw[e].y};
-      double2* dst = reinterpret_cast<double2*>(kst + e * DI + lane * 4);
-      dst[0] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[0] & 0xFFFFu)),
-                            bf16_to_f64(static_cast<uint16_t>(w[0] >> 16)));
-      dst[1] = make_double2(bf16_to_f64(static_cast<uint16_t>(w[1] & 0xFFFFu)),
-                            bf16_to_f64(static_cast<uint16_t>(w[1] >> 16)));
+      uint32_t h[4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        h[2 * u] = static_cast<uint32_t>(__double2hiint(bf16_to_f64(static_cast<uint16_t>(w[u] & 0xFFFFu))));
+        h[2 * u + 1] = static_cast<uint32_t>(__double2hiint(bf16_to_f64(static_cast<uint16_t>(w[u] >> 16))));
+      }
+      *reinterpret_cast<uint4*>(kst + e * DI + lane * 4) = make_uint4(h[0], h[1], h[2], h[3]);
     }
   }
   __syncwarp();
-  double pr[4] = {0.0, 0.0, 0.0, 0.0};
+  double pr[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) pr[e] = 0.0;
   if (lane < HI) {
     const uint4* q4 = reinterpret_cast<const uint4*>(qhi + lane * (DI + 4));
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+#pragma unroll 2
     for (int c4 = 0; c4 < DI / 4; ++c4) {
       const uint4 qq = q4[c4];
       const double qd[4] = {__hiloint2double(static_cast<int>(qq.x), 0), __hiloint2double(static_cast<int>(qq.y), 0),
                             __hiloint2double(static_cast<int>(qq.z), 0), __hiloint2double(static_cast<int>(qq.w), 0)};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const double2* kp = reinterpret_cast<const double2*>(kst + e * DI + c4 * 4);
-        const double2 k01 = kp[0], k23 = kp[1];
-        acc[e] = fma(qd[0], k01.x, acc[e]);
-        acc[e] = fma(qd[1], k01.y, acc[e]);
-        acc[e] = fma(qd[2], k23.x, acc[e]);
-        acc[e] = fma(qd[3], k23.y, acc[e]);
+      for (int e = 0; e < 8; ++e) {
+        const uint4 kk = reinterpret_cast<const uint4*>(kst + e * DI)[c4];
+        acc[e] = fma(qd[0], __hiloint2double(static_cast<int>(kk.x), 0), acc[e]);
+        acc[e] = fma(qd[1], __hiloint2double(static_cast<int>(kk.y), 0), acc[e]);
+        acc[e] = fma(qd[2], __hiloint2double(static_cast<int>(kk.z), 0), acc[e]);
+        acc[e] = fma(qd[3], __hiloint2double(static_cast<int>(kk.w), 0), acc[e]);
       }
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pr[e] = __dmul_rn(w_lane, acc[e] > 0.0 ? acc[e] : 0.0);
+    for (int e = 0; e < 8; ++e) pr[e] = __dmul_rn(w_lane, acc[e] > 0.0 ? acc[e] : 0.0);
   }
   __syncwarp();
-  double* prod = kst;
+  double* prod = reinterpret_cast<double*>(kst);
   if (lane < HI) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) prod[e * 34 + lane] = pr[e];
+    for (int e = 0; e < 8; ++e) prod[e * 34 + lane] = pr[e];
   }
   __syncwarp();
   double sum = 0.0;
-  if (lane < 4) {
+  if (lane < 8) {
     const double2* pe = reinterpret_cast<const double2*>(prod + lane * 34);
 #pragma unroll
     for (int j2 = 0; j2 < 16; ++j2) {
@@ -962,8 +966,12 @@ constexpr int kFThreads = 192;
 constexpr int kFWarps = kFThreads / 32;
 constexpr int kFChunk = 128;
 constexpr int kWinCap = 256;
-// hist (2,048 ints), or the re-score's key staging: 4 keys x 128 float64 per warp
-constexpr int kFRegionBytes = (kBins * 4 > kFWarps * 4 * 128 * 8) ? kBins * 4 : kFWarps * 4 * 128 * 8;
+// hist (2,048 ints), or the re-score's key staging: per warp 1,024 words,
+// eight keys of up to 128 dims as float64 high words and then the head sum's
+// [8][34] float64 products
+constexpr int kFKstWords = 1024;
+static_assert(kFKstWords >= 8 * 128 && kFKstWords * 4 >= 8 * 34 * 8, "window select key staging");
+constexpr int kFRegionBytes = (kBins * 4 > kFWarps * kFKstWords * 4) ? kBins * 4 : kFWarps * kFKstWords * 4;
 
 // kSeg: pass 1 of the long-row select (topk_kernel's pass 1): CTA (row,
 // segment) selects among the segment's keys key_off .. key_off + n - 1 and
@@ -1199,25 +1207,16 @@ __global__ void __launch_bounds__(kFThreads, 4) topk_window_kernel(TopkArgs a) {
         // re-score the band four keys per warp call (the next four key rows
         // are loaded while the current ones are scored)
         const double w_lane = lane < HI ? static_cast<double>(w_pre) : 0.0;
-        double* my_kst = kst_all + warp * 4 * DI;
-        int b = 4 * warp;
-        uint2 raw[4];
+        // (4 KB per warp: eight 128-dim keys, or the [8][34] float64 products)
+        uint32_t* my_kst = reinterpret_cast<uint32_t*>(kst_all) + warp * kFKstWords;
+        for (int b = 8 * warp; b < tot_band; b += 8 * kFWarps) {
+          uint2 raw[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          raw[e] = b < tot_band ? load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)] + key_off, DI)
-                                : make_uint2(0u, 0u);
-        for (; b < tot_band; b += 4 * kFWarps) {
-          const int bn = b + 4 * kFWarps;
-          uint2 nraw[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            nraw[e] = bn < tot_band ? load_key_part(a.k_idx, bidx[min(bn + e, tot_band - 1)] + key_off, DI)
-                                    : make_uint2(0u, 0u);
-          const double xl = rescore4d<DI>(qhi, w_lane, raw, my_kst, HI);
-          if (lane < 4 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, kWinCap, 52))
+          for (int e = 0; e < 8; ++e)
+            raw[e] = load_key_part(a.k_idx, bidx[min(b + e, tot_band - 1)] + key_off, DI);
+          const double xl = rescore8h<DI>(qhi, w_lane, raw, my_kst, HI);
+          if (lane < 8 && b + lane < tot_band && DSA_IN_BOUNDS(a.ws, b + lane, kWinCap, 52))
             bx[b + lane] = d2key(xl);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) raw[e] = nraw[e];
         }
         __syncthreads();
         // rank by (X desc, key asc): a warp takes four band keys at a time
