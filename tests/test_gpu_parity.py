@@ -211,18 +211,23 @@ def test_topk_exact_mode_on_gpu_scores(dsa, oracle_lib):
     assert np.array_equal(idx.cpu().numpy(), ref)
 
 
-@pytest.mark.parametrize("T", [
-    18400,   # two CTAs per SM, eight re-scoring warps, a smaller band cache
-    30000,   # one CTA per SM
-])
-def test_topk_exact_mode_launch_variants(dsa, oracle_lib, T):
-    """The top-k launch picks its shared-memory layout by context length; each
-    layout reproduces the float64 order."""
+@pytest.mark.parametrize("T,kind", [
+    (18400, "normal"),          # the window select
+    (30000, "normal"),
+    (18400, "repeated_keys"),   # 40 distinct key rows: every score ties with hundreds of others,
+    (30000, "repeated_keys"),   # the window overflows and the rows are handed back to the bucket
+])                              # select (two CTAs per SM at 18,400 keys, one at 30,000)
+def test_topk_exact_mode_launch_variants(dsa, oracle_lib, T, kind):
+    """The exact mode's kernels and shared-memory layouts by context length:
+    the window select, and the bucket select on the rows it hands back; each
+    reproduces the float64 order."""
     import torch
 
     n_q = 6
     d = make_dims(n_q, T - n_q, T, 32, 512, 64, 32, 128, 2048)
     x = workloads.generate(d, 31, "normal", "uniform")
+    if kind == "repeated_keys":
+        x["k_idx"] = np.ascontiguousarray(x["k_idx"][np.arange(T) % 40])
     xd = stage(x)
     ld = (T + 3) // 4 * 4
     sc = torch.empty(d.n_q, ld, dtype=torch.float32, device="cuda")
@@ -230,9 +235,15 @@ def test_topk_exact_mode_launch_variants(dsa, oracle_lib, T):
     dsa.check(dsa.dsa_index_scores(d, xd["q_idx"], xd["k_idx"], xd["w_idx"], sc, ld, ws))
     idx = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
     dsa.check(dsa.dsa_topk_select(d, sc, ld, xd["q_idx"], xd["k_idx"], xd["w_idx"], idx, ws))
+    torch.cuda.synchronize()
+    # the workspace header counts the rows the window select handed back
+    # (a 32-bit word at byte 24)
+    handed_back = int(ws[24:28].cpu().numpy().view(np.uint32)[0])
     dsa.check(dsa.dsa_device_status(ws))
     ref = oracle_lib.topk_select(d, oracle_lib.index_scores(d, x["q_idx"], x["k_idx"], x["w_idx"]))
     assert np.array_equal(idx.cpu().numpy(), ref)
+    if kind == "repeated_keys":
+        assert handed_back > 0
 
 
 @pytest.mark.parametrize("n_q,n_sub", [
