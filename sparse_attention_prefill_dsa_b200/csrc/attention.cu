@@ -275,7 +275,7 @@ struct AttnBars {
   static_assert(kCount == C::kNumBars, "barrier count");
 };
 
-// A wait by every lane of a warp, with one verdict for the whole warp.
+// A wait by every lane of a warp, with one outcome for the whole warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           WsHeader* ws, unsigned site) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, ws, site));
