@@ -102,6 +102,7 @@ typedef int32_t dsa_status;
 #define DSA_ERR_RANGE (-9)     /* device found a selected index outside 0..t           */
 #define DSA_ERR_SCRATCH_LIMIT (-10) /* dsa_prefill_layer_noalloc: the chunk needs more
                                        scratch than DSA_NOALLOC_SCRATCH_BYTES             */
+#define DSA_ERR_LAYOUT (-11)   /* dsa_selftest_mma_layout: a tensor-core product differed */
 
 /* Which call a workspace is for. */
 #define DSA_WS_INDEX_SCORES 0
@@ -392,8 +393,35 @@ dsa_status dsa_partition_queries(const dsa_dims* dims, int32_t n_parts, int32_t*
 dsa_status dsa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, int64_t* cycles,
                                      void* stream);
 
+/* Start-up self-test of the tensor-core operand layouts the kernels use (the
+ * TensorFold issue #743 page, "Pre-M5 kernel checks": a load-time check of the
+ * matrix-fragment layout that a transposed operand got through). One CTA
+ * multiplies small-integer matrices that are not symmetric, each laid out in
+ * shared memory as the kernels' own copies lay it out and multiplied with the
+ * kernels' descriptor conventions, and compares every accumulator element
+ * with a sum of the same integers on the CUDA cores; both are exact in
+ * float32, so any difference means a transposed operand or a wrong swizzle,
+ * stride, descriptor field or tensor-memory mapping. Forms, in order:
+ *   0 the indexer's bf16 MMA (M 128, N 256, K 128, K-major, 128-byte swizzle)
+ *   1 the attention's QK^T (M 128 keys, N 32 heads, K-major)
+ *   2 the attention's PV (latent pair read MN-major, P in 64-byte swizzled
+ *     rows, N 32)
+ *   3 the FP8 indexer's e4m3 MMA (kind::f8f6f4, M 128, N 256, K 128)
+ *   workspace   >= 272 bytes (16-byte aligned); its header is cleared first,
+ *               and bytes 256..271 receive the four counts on the device
+ *   mismatches  host int32 [4] (may be NULL): wrong accumulator elements of
+ *               each form (all 0 when the layouts hold; -1 when an MMA did
+ *               not complete within the kernels' wait limit). When given,
+ *               the call synchronizes `stream` and copies the counts back.
+ * A wrong element also records DSA_ERR_LAYOUT (site = the first bad form) in
+ * the workspace status, read by dsa_device_status. Run it once per device
+ * before the first layer call. Errors: DSA_ERR_WORKSPACE, _ALIGN, _DEVICE,
+ * _CUDA. */
+dsa_status dsa_selftest_mma_layout(void* workspace, size_t workspace_bytes, int32_t* mismatches,
+                                   void* stream);
+
 /* Synchronizes `stream`, returns the device status word of `workspace`
- * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_RANGE) and clears it. */
+ * (DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_RANGE or DSA_ERR_LAYOUT) and clears it. */
 dsa_status dsa_device_status(void* workspace, void* stream);
 
 /* Static text for a status code. */

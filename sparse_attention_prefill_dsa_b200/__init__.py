@@ -36,6 +36,7 @@ DSA_ERR_CUDA = -7
 DSA_ERR_DEVICE = -8
 DSA_ERR_RANGE = -9
 DSA_ERR_SCRATCH_LIMIT = -10
+DSA_ERR_LAYOUT = -11
 DSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 DSA_WS_INDEX_SCORES = 0
@@ -58,7 +59,7 @@ EXPORTED = ("dsa_workspace_size", "dsa_index_scores", "dsa_topk_select",
             "dsa_status_string", "dsa_prefill_layer_noalloc", "dsa_prefill_layer_host",
             "dsa_selftest_bounded_wait", "dsa_partition_queries", "dsa_sparse_attn_decode",
             "dsa_decode_layer", "dsa_sparse_attn_block", "dsa_quantize_fp8",
-            "dsa_index_scores_fp8")
+            "dsa_index_scores_fp8", "dsa_selftest_mma_layout")
 
 
 class dsa_dims(ctypes.Structure):
@@ -123,6 +124,7 @@ def library():
                                            ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
                                            ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int32]
     lib.dsa_selftest_bounded_wait.argtypes = [_P, ctypes.c_size_t, _P, _P]
+    lib.dsa_selftest_mma_layout.argtypes = [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32), _P]
     lib.dsa_partition_queries.argtypes = [_DP, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     lib.dsa_device_status.argtypes = [_P, _P]
     lib.dsa_status_string.argtypes = [ctypes.c_int32]
@@ -131,7 +133,7 @@ def library():
               "dsa_prefill_layer", "dsa_device_status", "dsa_prefill_layer_noalloc",
               "dsa_prefill_layer_host", "dsa_selftest_bounded_wait", "dsa_partition_queries",
               "dsa_sparse_attn_decode", "dsa_decode_layer", "dsa_sparse_attn_block",
-              "dsa_quantize_fp8", "dsa_index_scores_fp8"):
+              "dsa_quantize_fp8", "dsa_index_scores_fp8", "dsa_selftest_mma_layout"):
         getattr(lib, f).restype = ctypes.c_int32
     _lib = lib
     return lib
@@ -269,6 +271,15 @@ def dsa_selftest_bounded_wait(workspace, cycles=None, workspace_bytes=None, stre
     optional device int64 tensor of 2 elements."""
     return library().dsa_selftest_bounded_wait(_p(workspace), _nbytes(workspace, workspace_bytes),
                                                _p(cycles), _stream(stream))
+
+
+def dsa_selftest_mma_layout(workspace, workspace_bytes=None, stream=None):
+    """The tensor-core layout self-test (see include/dsa.h): returns (status,
+    [wrong elements of each of the four forms])."""
+    counts = (ctypes.c_int32 * 4)()
+    st = library().dsa_selftest_mma_layout(_p(workspace), _nbytes(workspace, workspace_bytes),
+                                           counts, _stream(stream))
+    return st, list(counts)
 
 
 def dsa_device_status(workspace, stream=None) -> int:

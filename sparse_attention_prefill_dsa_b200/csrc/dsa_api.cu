@@ -510,6 +510,26 @@ dsa_status dsa_selftest_bounded_wait(void* ws, size_t ws_bytes, int64_t* cycles,
                                                      reinterpret_cast<long long*>(cycles), st));
 }
 
+dsa_status dsa_selftest_mma_layout(void* ws, size_t ws_bytes, int32_t* mismatches, void* stream) {
+  if (!ws || ws_bytes < dsa::kWsHeaderBytes + 16) return DSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return DSA_ERR_ALIGN;
+  dsa_status s = check_device();
+  if (s != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_header(ws, st)) != DSA_OK) return s;
+  int* dev_counts = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + dsa::kWsHeaderBytes);
+  if ((s = from_cuda(dsa::launch_mma_layout_selftest(static_cast<dsa::WsHeader*>(ws), dev_counts,
+                                                     st))) != DSA_OK)
+    return s;
+  if (mismatches) {
+    if (cudaMemcpyAsync(mismatches, dev_counts, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
 dsa_status dsa_device_status(void* ws, void* stream) {
   if (!ws) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -521,6 +541,7 @@ dsa_status dsa_device_status(void* ws, void* stream) {
     return DSA_ERR_CUDA;
   if (code == dsa::kDevTimeout) return DSA_ERR_TIMEOUT;
   if (code == dsa::kDevRange) return DSA_ERR_RANGE;
+  if (code == dsa::kDevLayout) return DSA_ERR_LAYOUT;
   return code == 0 ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -536,6 +557,8 @@ const char* dsa_status_string(dsa_status s) {
     case DSA_ERR_CUDA: return "CUDA runtime or launch error";
     case DSA_ERR_DEVICE: return "current device is not an sm_100 (B200) GPU";
     case DSA_ERR_RANGE: return "a selected index was outside the causal range 0..t of its query";
+    case DSA_ERR_LAYOUT:
+      return "the tensor-core layout self-test found an accumulator element that differs";
     case DSA_ERR_SCRATCH_LIMIT:
       return "the chunk needs more scratch than the no-alloc entry point's static array holds";
     default: return "unknown status";

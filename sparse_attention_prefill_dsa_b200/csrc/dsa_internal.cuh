@@ -10,7 +10,7 @@ namespace dsa {
 
 // First 256 bytes of every workspace.
 struct WsHeader {
-  unsigned int status;        // 0 or a positive code: kDevTimeout / kDevRange
+  unsigned int status;        // 0 or a positive code: kDevTimeout / kDevRange / ...
   unsigned int status_info;   // first failing site (kernel-specific)
   unsigned long long kmax_bits;  // float64 bit pattern of max_s ||k_idx[s]||_2 (>= 0)
   unsigned int akmax_bits;       // float32 bit pattern of max_s ||[latent_s, rope_s]||_2 (>= 0)
@@ -23,6 +23,7 @@ static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 constexpr unsigned int kDevTimeout = 1;
 constexpr unsigned int kDevRange = 2;
 constexpr unsigned int kDevInternal = 3;  // an internal consistency check failed
+constexpr unsigned int kDevLayout = 4;    // the tensor-core layout self-test found a wrong element
 // wait sites of the bounded-wait self-test (the kernels use sites below 100)
 constexpr unsigned int kSelftestSiteShort = 101;
 constexpr unsigned int kSelftestSiteLong = 102;
@@ -134,5 +135,6 @@ cudaError_t launch_block_attn(const dsa_dims& d, const uint16_t* q, const uint16
 
 // The bounded-wait self-test (one CTA, two warps on mbarriers nothing signals).
 cudaError_t launch_bounded_wait_selftest(WsHeader* ws, long long* cycles, cudaStream_t st);
+cudaError_t launch_mma_layout_selftest(WsHeader* ws, int* mismatches, cudaStream_t st);
 
 }  // namespace dsa

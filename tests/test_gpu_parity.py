@@ -391,6 +391,17 @@ def test_bounded_wait_gives_up_cleanly(dsa, oracle_lib):
     _compare_layer(oracle_lib, d, x, out, lse, idx)
 
 
+def test_mma_layout_selftest_passes(dsa):
+    """The start-up check of the tensor-core operand layouts: every accumulator
+    element of the four forms (indexer bf16, attention QK^T and PV, FP8
+    indexer) equals the exact integer product, and nothing is reported."""
+    ws = workspace(512)
+    st, counts = dsa.dsa_selftest_mma_layout(ws)
+    dsa.check(st)
+    assert counts == [0, 0, 0, 0]
+    assert dsa.dsa_device_status(ws) == dsa.DSA_OK
+
+
 def test_empty_chunk_launches_nothing(dsa):
     import torch
 
