@@ -12,7 +12,7 @@
 // w-weighted head sum and the store with no cross-thread traffic, and a warp
 // writes 32 consecutive keys of a query row (128 coalesced bytes).
 //
-// Persistent, warp-specialised CTA (one per SM, 320 threads):
+// Persistent, warp-specialised CTA (one per SM, 576 threads):
 //   warp 0      TMA producer: takes work units from a queue (an atomic
 //               counter in the workspace header, reset before each launch),
 //               hands each unit to the other warps through a four-slot ring
@@ -24,8 +24,11 @@
 //               -> f32), issued warp-collectively by one elected lane with
 //               base descriptors plus compile-time offsets, accumulating each
 //               tile into one of two 256-column TMEM buffers;
-//   warps 2-9   epilogue: two warpgroups split the 256 columns; each thread
-//               reads its key's columns with tcgen05.ld and writes the scores.
+//   warps 2-17  epilogue: four warpgroups split the 256 columns (64 each);
+//               each thread reads its key's columns with tcgen05.ld, hands
+//               the accumulator buffer back as soon as they are in registers
+//               (the next tile but one accumulates there while this one is
+//               summed), and writes the scores.
 // A work unit is (query block, up to 32 consecutive causal key tiles). The
 // queue hands units out in slot-major order with the later (longer) query
 // blocks first, so every block's first 32 tiles go out before any block's
@@ -74,7 +77,10 @@ struct IdxCfg {
   static constexpr int kKSteps = DI / kKPerMma;
   static constexpr int kStepsPerChunk = kChunk / kKPerMma;
   static constexpr int kTilesPerUnit = 32;             // key tiles per work unit (fewer for small chunks)
-  static constexpr int kEpiWarps = 8;                  // warps 2-9
+  static constexpr int kEpiWarps = 16;                 // warps 2-17: four per TMEM lane quarter
+  static constexpr int kEpiGroups = kEpiWarps / 4;     // column ranges, one per warpgroup
+  static constexpr int kColsPerWg = kN / kEpiGroups;   // accumulator columns per epilogue warp
+  static constexpr int kGroups = kColsPerWg / 32;      // 32-column TMEM loads per tile and warp
   static constexpr int kThreads = 32 * (2 + kEpiWarps);
   static constexpr uint32_t kIdesc = FP8 ? idesc_e4m3_f32(kM, kN) : idesc_bf16_f32(kM, kN, false, false);
   // shared memory carve (offsets from a 1024-byte aligned base)
@@ -322,7 +328,7 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI, FP8>::kThreads, 1)
     drain_wait(mma_done, 0);
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 2) >> 2;        // column half
+    const int wg = (warp - 2) >> 2;        // column range (kColsPerWg columns)
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int key_local = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -347,66 +353,57 @@ __global__ void __launch_bounds__(IdxCfg<HI, DI, FP8>::kThreads, 1)
         // FP8: the key row's scale, applied to the finished head sum (a power
         // of two: relu(s_k x) = s_k relu(x), and the product is exact)
         const float ks = FP8 ? (s < p.ctx_len ? __ldg(p.k_scale + s) : 0.f) : 1.f;
-        // four 32-column groups, two per TMEM wait; with 32 heads the loads of
-        // the next two groups are in flight while the current two are summed
-        // (with 2 heads a group holds 16 queries and the registers would not
-        // hold four). The weights of a group are read as float4 broadcasts.
-        constexpr bool kAhead = HI == 32;
-        uint32_t v[4][32];
+        // the warp's 32-column groups: all loaded, and the accumulator handed
+        // back to the MMA warp as soon as they are in registers, so the next
+        // tile but one accumulates there while this one is summed
+        uint32_t v[C::kGroups][32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + h * 32, v[h]);
+        for (int h = 0; h < C::kGroups; ++h)
+          tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * C::kColsPerWg + h * 32, v[h]);
         tmem_ld_wait();
-#pragma unroll
-        for (int g2 = 0; g2 < 2; ++g2) {
-          if (g2 == 0 && kAhead) {
-#pragma unroll
-            for (int h = 2; h < 4; ++h)
-              tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + h * 32, v[h]);
-          } else if (g2 == 1) {
-            if (!kAhead) {
-#pragma unroll
-              for (int h = 2; h < 4; ++h)
-                tmem_ld_32x32b_x32(tmem_base + lane_addr + buf * C::kN + wg * 128 + h * 32, v[h]);
-            }
-            tmem_ld_wait();
-          }
-#pragma unroll
-          for (int h = 2 * g2; h < 2 * g2 + 2; ++h) {
-            const int col0 = wg * 128 + h * 32;
-            float wv[32];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float4 w4 = *reinterpret_cast<const float4*>(w + col0 + 4 * e);
-              wv[4 * e] = w4.x;
-              wv[4 * e + 1] = w4.y;
-              wv[4 * e + 2] = w4.z;
-              wv[4 * e + 3] = w4.w;
-            }
-#pragma unroll
-            for (int qq = 0; qq < 32 / HI; ++qq) {
-              // the head sum in four interleaved partial sums (heads j mod 4),
-              // so that consecutive multiply-adds do not wait on each other
-              constexpr int kPart = HI >= 4 ? 4 : HI;
-              float part[kPart];
-#pragma unroll
-              for (int u = 0; u < kPart; ++u) part[u] = 0.f;
-#pragma unroll
-              for (int j = 0; j < HI; ++j)
-                part[j % kPart] = fmaf(wv[qq * HI + j], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f),
-                                       part[j % kPart]);
-              float acc = part[0];
-#pragma unroll
-              for (int u = 1; u < kPart; ++u) acc += part[u];
-              const int i = qb * C::kQB + (col0 + qq * HI) / HI;
-              if (i < p.n_q && s <= p.q_pos0 + i && DSA_IN_BOUNDS(p.ws, s, p.ld, 20))
-                p.scores[static_cast<int64_t>(i) * p.ld + s] = FP8 ? acc * ks : acc;
-            }
-          }
-        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+        for (int h = 0; h < C::kGroups; ++h) {
+          const int col0 = wg * C::kColsPerWg + h * 32;
+#pragma unroll
+          for (int qq = 0; qq < 32 / HI; ++qq) {
+            // the head sum in four interleaved partial sums (heads j mod 4),
+            // so that consecutive multiply-adds do not wait on each other;
+            // the weights are read as float4 broadcasts
+            constexpr int kPart = HI >= 4 ? 4 : HI;
+            float part[kPart];
+#pragma unroll
+            for (int u = 0; u < kPart; ++u) part[u] = 0.f;
+#pragma unroll
+            for (int j0 = 0; j0 < HI; j0 += 4) {
+              float wv[4];
+              if constexpr (HI >= 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(w + col0 + qq * HI + j0);
+                wv[0] = w4.x;
+                wv[1] = w4.y;
+                wv[2] = w4.z;
+                wv[3] = w4.w;
+              } else {
+#pragma unroll
+                for (int e = 0; e < HI; ++e) wv[e] = w[col0 + qq * HI + e];
+              }
+#pragma unroll
+              for (int e = 0; e < 4 && j0 + e < HI; ++e) {
+                const int j = j0 + e;
+                part[j % kPart] = fmaf(wv[e], fmaxf(__uint_as_float(v[h][qq * HI + j]), 0.f),
+                                       part[j % kPart]);
+              }
+            }
+            float acc = part[0];
+#pragma unroll
+            for (int u = 1; u < kPart; ++u) acc += part[u];
+            const int i = qb * C::kQB + (col0 + qq * HI) / HI;
+            if (i < p.n_q && s <= p.q_pos0 + i && DSA_IN_BOUNDS(p.ws, s, p.ld, 20))
+              p.scores[static_cast<int64_t>(i) * p.ld + s] = FP8 ? acc * ks : acc;
+          }
+        }
       }
       if (!ok) break;
       __syncwarp();
