@@ -407,18 +407,23 @@ dsa_status dsa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, in
  *   2 the attention's PV (latent pair read MN-major, P in 64-byte swizzled
  *     rows, N 32)
  *   3 the FP8 indexer's e4m3 MMA (kind::f8f6f4, M 128, N 256, K 128)
- *   workspace   >= 272 bytes (16-byte aligned); its header is cleared first,
- *               and bytes 256..271 receive the four counts on the device
+ *   workspace   >= 288 bytes (16-byte aligned); its header is cleared first;
+ *               bytes 256..271 receive the four counts and 272..287 the four
+ *               timings on the device
  *   mismatches  host int32 [4] (may be NULL): wrong accumulator elements of
  *               each form (all 0 when the layouts hold; -1 when an MMA did
- *               not complete within the kernels' wait limit). When given,
- *               the call synchronizes `stream` and copies the counts back.
+ *               not complete within the kernels' wait limit)
+ *   cycles_per_mma  host float [4] (may be NULL): each form's MMAs issued 32
+ *               times back to back on one SM, SM clock cycles per MMA from
+ *               the first issue to the last completion (-1 as above)
+ * When either host array is given, the call synchronizes `stream` and copies
+ * the results back.
  * A wrong element also records DSA_ERR_LAYOUT (site = the first bad form) in
  * the workspace status, read by dsa_device_status. Run it once per device
  * before the first layer call. Errors: DSA_ERR_WORKSPACE, _ALIGN, _DEVICE,
  * _CUDA. */
 dsa_status dsa_selftest_mma_layout(void* workspace, size_t workspace_bytes, int32_t* mismatches,
-                                   void* stream);
+                                   float* cycles_per_mma, void* stream);
 
 /* Synchronizes `stream`, returns the device status word of `workspace`
  * (DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_RANGE or DSA_ERR_LAYOUT) and clears it. */

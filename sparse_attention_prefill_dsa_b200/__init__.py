@@ -124,7 +124,8 @@ def library():
                                            ctypes.POINTER(dsa_device_tensors), _P, ctypes.c_size_t,
                                            ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int32]
     lib.dsa_selftest_bounded_wait.argtypes = [_P, ctypes.c_size_t, _P, _P]
-    lib.dsa_selftest_mma_layout.argtypes = [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32), _P]
+    lib.dsa_selftest_mma_layout.argtypes = [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32),
+                                            ctypes.POINTER(ctypes.c_float), _P]
     lib.dsa_partition_queries.argtypes = [_DP, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     lib.dsa_device_status.argtypes = [_P, _P]
     lib.dsa_status_string.argtypes = [ctypes.c_int32]
@@ -275,11 +276,12 @@ def dsa_selftest_bounded_wait(workspace, cycles=None, workspace_bytes=None, stre
 
 def dsa_selftest_mma_layout(workspace, workspace_bytes=None, stream=None):
     """The tensor-core layout self-test (see include/dsa.h): returns (status,
-    [wrong elements of each of the four forms])."""
+    [wrong elements of each of the four forms], [cycles per MMA of each form])."""
     counts = (ctypes.c_int32 * 4)()
+    cycles = (ctypes.c_float * 4)()
     st = library().dsa_selftest_mma_layout(_p(workspace), _nbytes(workspace, workspace_bytes),
-                                           counts, _stream(stream))
-    return st, list(counts)
+                                           counts, cycles, _stream(stream))
+    return st, list(counts), list(cycles)
 
 
 def dsa_device_status(workspace, stream=None) -> int:

@@ -510,23 +510,29 @@ dsa_status dsa_selftest_bounded_wait(void* ws, size_t ws_bytes, int64_t* cycles,
                                                      reinterpret_cast<long long*>(cycles), st));
 }
 
-dsa_status dsa_selftest_mma_layout(void* ws, size_t ws_bytes, int32_t* mismatches, void* stream) {
-  if (!ws || ws_bytes < dsa::kWsHeaderBytes + 16) return DSA_ERR_WORKSPACE;
+dsa_status dsa_selftest_mma_layout(void* ws, size_t ws_bytes, int32_t* mismatches,
+                                   float* cycles_per_mma, void* stream) {
+  if (!ws || ws_bytes < dsa::kWsHeaderBytes + 32) return DSA_ERR_WORKSPACE;
   if (!aligned16(ws)) return DSA_ERR_ALIGN;
   dsa_status s = check_device();
   if (s != DSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = clear_header(ws, st)) != DSA_OK) return s;
-  int* dev_counts = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + dsa::kWsHeaderBytes);
+  unsigned char* out = static_cast<unsigned char*>(ws) + dsa::kWsHeaderBytes;
+  int* dev_counts = reinterpret_cast<int*>(out);
+  float* dev_cycles = reinterpret_cast<float*>(out + 16);
   if ((s = from_cuda(dsa::launch_mma_layout_selftest(static_cast<dsa::WsHeader*>(ws), dev_counts,
-                                                     st))) != DSA_OK)
+                                                     dev_cycles, st))) != DSA_OK)
     return s;
-  if (mismatches) {
-    if (cudaMemcpyAsync(mismatches, dev_counts, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
-            cudaSuccess ||
-        cudaStreamSynchronize(st) != cudaSuccess)
-      return DSA_ERR_CUDA;
-  }
+  if (mismatches &&
+      cudaMemcpyAsync(mismatches, dev_counts, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (cycles_per_mma &&
+      cudaMemcpyAsync(cycles_per_mma, dev_cycles, 4 * sizeof(float), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return DSA_ERR_CUDA;
+  if ((mismatches || cycles_per_mma) && cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }
 

@@ -135,6 +135,7 @@ cudaError_t launch_block_attn(const dsa_dims& d, const uint16_t* q, const uint16
 
 // The bounded-wait self-test (one CTA, two warps on mbarriers nothing signals).
 cudaError_t launch_bounded_wait_selftest(WsHeader* ws, long long* cycles, cudaStream_t st);
-cudaError_t launch_mma_layout_selftest(WsHeader* ws, int* mismatches, cudaStream_t st);
+cudaError_t launch_mma_layout_selftest(WsHeader* ws, int* mismatches, float* cycles_per_mma,
+                                      cudaStream_t st);
 
 }  // namespace dsa

@@ -22,6 +22,9 @@
 //   form 3  FP8 indexer: e4m3 operands [128][128] and [256][128] in 128-byte
 //           rows, kind::f8f6f4, 4 MMAs of K = 32.
 // Results read back with tcgen05.ld 32x32b (thread = accumulator row).
+// Each form is then timed: its MMAs issued 32 times back to back on the same
+// operands, clock64 from the first issue to the completion of the last, which
+// gives the form's cycles per MMA on one SM.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,6 +42,7 @@ constexpr int kOperandBytes = 96 * 1024;  // form 0: A 32 KB + B 64 KB
 constexpr int kOffB = 32 * 1024;
 constexpr int kSmemBytes = kOperandBytes + 64 + 1024;  // + barrier and counters, alignment slack
 constexpr unsigned int kSiteMma = 103;     // the wait for a form's MMAs
+constexpr int kTimedReps = 32;             // repetitions of a form's MMAs in its timed run
 
 // The test matrices: small integers from a hash of (row, column), exact in
 // bf16 and e4m3, with products and 128-term sums exact in float32; no two
@@ -111,10 +115,12 @@ __device__ void fill_form(int form, unsigned char* s) {
   }
 }
 
-// Issues the form's MMAs into tensor-memory column 0 (warp-collective).
-__device__ void issue_form(int form, unsigned char* s, uint32_t tmem) {
+// Issues the form's MMAs into tensor-memory column 0 (warp-collective), with
+// the descriptors as compile-time offsets from two bases, as the kernels do.
+template <int form>
+__device__ __forceinline__ void issue_form(unsigned char* s, uint32_t tmem) {
   const uint32_t a0 = smem_u32(s), b0 = smem_u32(s + kOffB);
-  if (form == 0) {
+  if constexpr (form == 0) {
     const uint64_t da = smem_desc(a0, 16, 1024, 2), db = smem_desc(b0, 16, 1024, 2);
     constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, false);
 #pragma unroll
@@ -123,7 +129,7 @@ __device__ void issue_form(int form, unsigned char* s, uint32_t tmem) {
       mma_bf16_ss_warp(tmem, da + ((c * 16384 + off) >> 4), db + ((c * 32768 + off) >> 4), idesc,
                        ks > 0 ? 1u : 0u);
     }
-  } else if (form == 1) {
+  } else if constexpr (form == 1) {
     const uint64_t da = smem_desc(a0, 16, 1024, 2), db = smem_desc(b0, 16, 1024, 2);
     constexpr uint32_t idesc = idesc_bf16_f32(128, 32, false, false);
 #pragma unroll
@@ -132,7 +138,7 @@ __device__ void issue_form(int form, unsigned char* s, uint32_t tmem) {
       for (int ks = 0; ks < 4; ++ks)
         mma_bf16_ss_warp(tmem, da + ((c * 16384 + ks * 32) >> 4), db + ((c * 4096 + ks * 32) >> 4),
                          idesc, (c | ks) ? 1u : 0u);
-  } else if (form == 2) {
+  } else if constexpr (form == 2) {
     const uint64_t da = smem_desc(a0, 16384, 1024, 2), db = smem_desc(b0, 8 * 64, 8 * 64, 4);
     constexpr uint32_t idesc = idesc_bf16_f32(128, 32, true, true);
 #pragma unroll
@@ -148,7 +154,26 @@ __device__ void issue_form(int form, unsigned char* s, uint32_t tmem) {
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) mma_layout_selftest(WsHeader* ws, int* mismatches) {
+__device__ __forceinline__ int mmas_of_form(int form) { return form == 3 ? 4 : 8; }
+
+// The form's MMAs once (reps = 1) or kTimedReps times back to back (warp-collective).
+template <int form>
+__device__ __forceinline__ void issue_reps(unsigned char* s, uint32_t tmem, int reps) {
+#pragma unroll 1
+  for (int r = 0; r < reps; ++r) issue_form<form>(s, tmem);
+}
+
+__device__ __forceinline__ void issue_form_n(int form, unsigned char* s, uint32_t tmem, int reps) {
+  switch (form) {
+    case 0: issue_reps<0>(s, tmem, reps); break;
+    case 1: issue_reps<1>(s, tmem, reps); break;
+    case 2: issue_reps<2>(s, tmem, reps); break;
+    default: issue_reps<3>(s, tmem, reps); break;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mma_layout_selftest(WsHeader* ws, int* mismatches,
+                                                                   float* cycles_per_mma) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* s = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -171,18 +196,19 @@ __global__ void __launch_bounds__(kThreads, 1) mma_layout_selftest(WsHeader* ws,
   const uint32_t tmem = *tmem_slot;
   const int m = 32 * warp + lane;  // this thread's accumulator row (tensor-memory lane)
   bool ok = true;
-  int issued = 0;
+  uint32_t phase = 0;  // commits made to `bar`
+  float s_cyc[kForms] = {0.f, 0.f, 0.f, 0.f};
   for (int form = 0; form < kForms && ok; ++form) {
     fill_form(form, s);
     fence_proxy_async_smem();  // generic-proxy writes, read by the MMAs through the async proxy
     __syncthreads();
     if (warp == 0) {
       tc_fence_after();
-      issue_form(form, s, tmem);
+      issue_form_n(form, s, tmem, 1);
       mma_commit_warp(bar);
     }
-    ++issued;
-    ok = __all_sync(0xffffffffu, mbar_wait(bar, form & 1, abort_flag, ws, kSiteMma));
+    ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1, abort_flag, ws, kSiteMma));
+    ++phase;
     if (!ok) break;
     tc_fence_after();
     const int n_cols = (form == 1 || form == 2) ? 32 : 256;
@@ -200,12 +226,26 @@ __global__ void __launch_bounds__(kThreads, 1) mma_layout_selftest(WsHeader* ws,
     }
     if (bad) atomicAdd(&s_mis[form], bad);
     tc_fence_before();
-    __syncthreads();  // every thread has read the accumulator before the next form's MMAs
+    __syncthreads();  // every thread has read the accumulator before the timed MMAs
+    if (warp == 0) {
+      tc_fence_after();
+      const long long t0 = clock64();
+      issue_form_n(form, s, tmem, kTimedReps);
+      mma_commit_warp(bar);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1, abort_flag, ws, kSiteMma));
+      const long long t1 = clock64();
+      s_cyc[form] = static_cast<float>(t1 - t0) / static_cast<float>(kTimedReps * mmas_of_form(form));
+    }
+    ++phase;
+    // every thread reaches this barrier (no short circuit): it also keeps the
+    // next form's operand writes behind the timed MMAs
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    tc_fence_after();
   }
   if (!ok) {
     // a wait gave up: let the MMAs in flight finish (bounded) before TMEM is released
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, (issued - 1) & 1))
+    while (phase > 0 && !mbar_try_wait(bar, (phase - 1) & 1))
       if (clock64() - t0 > kWaitLimitCycles) break;
   }
   __syncthreads();
@@ -213,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_layout_selftest(WsHeader* ws,
     int first_bad = -1;
     for (int f = 0; f < kForms; ++f) {
       mismatches[f] = ok ? s_mis[f] : -1;
+      cycles_per_mma[f] = ok ? s_cyc[f] : -1.f;
       if (ok && s_mis[f] != 0 && first_bad < 0) first_bad = f;
     }
     if (first_bad >= 0) report(ws, kDevLayout, static_cast<unsigned int>(first_bad));
@@ -225,11 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1) mma_layout_selftest(WsHeader* ws,
 
 }  // namespace
 
-cudaError_t launch_mma_layout_selftest(WsHeader* ws, int* mismatches, cudaStream_t st) {
+cudaError_t launch_mma_layout_selftest(WsHeader* ws, int* mismatches, float* cycles_per_mma,
+                                      cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(mma_layout_selftest,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  mma_layout_selftest<<<1, kThreads, kSmemBytes, st>>>(ws, mismatches);
+  mma_layout_selftest<<<1, kThreads, kSmemBytes, st>>>(ws, mismatches, cycles_per_mma);
   return cudaGetLastError();
 }
 

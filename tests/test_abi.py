@@ -131,9 +131,9 @@ def test_host_validation_before_any_device_call(dsa):
 
 def test_layout_selftest_validates_its_workspace_first(dsa):
     FAKE = 1 << 20
-    st, counts = dsa.dsa_selftest_mma_layout(None, 0, 0)
+    st, counts, cycles = dsa.dsa_selftest_mma_layout(None, 0, 0)
     assert st == dsa.DSA_ERR_WORKSPACE
-    assert dsa.dsa_selftest_mma_layout(FAKE, 271, 0)[0] == dsa.DSA_ERR_WORKSPACE  # header + 16
+    assert dsa.dsa_selftest_mma_layout(FAKE, 287, 0)[0] == dsa.DSA_ERR_WORKSPACE  # header + 32
     assert dsa.dsa_selftest_mma_layout(FAKE + 8, 4096, 0)[0] == dsa.DSA_ERR_ALIGN
 
 
