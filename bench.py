@@ -315,6 +315,8 @@ def run_ours(args):
     x = workloads.generate(d, rank_seed(wl.seed, rank), wl.kind, w_mode)
     if args.fp8_indexer:  # the FP8 indexer variant of the layer (its own selection contract)
         d = dataclasses.replace(d, flags=dsa.DSA_FLAG_FP8_INDEXER)
+    if args.l2_scores:  # the layer's scores and selection over L2-resident query sub-blocks
+        d = dataclasses.replace(d, flags=d.flags | dsa.DSA_FLAG_L2_SCORES)
     stream = torch.cuda.current_stream()
 
     def to_dev_bf16(a):
@@ -325,7 +327,11 @@ def run_ours(args):
     out = torch.empty(d.n_q, d.n_heads, d.d_latent, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(d.n_q, d.n_heads, dtype=torch.float32, device="cuda")
     idx = torch.empty(d.n_q, d.top_k, dtype=torch.int32, device="cuda")
-    ws_layer = torch.empty(dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER), dtype=torch.uint8,
+    # (sized for the whole-chunk schedule too: the end-to-end leg's host call uses it)
+    ws_layer = torch.empty(max(dsa.dsa_workspace_size(d, dsa.DSA_WS_LAYER),
+                               dsa.dsa_workspace_size(dataclasses.replace(
+                                   d, flags=d.flags & ~dsa.DSA_FLAG_L2_SCORES), dsa.DSA_WS_LAYER)),
+                           dtype=torch.uint8,
                            device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
@@ -443,7 +449,8 @@ def run_ours(args):
     set_free = [torch.cuda.Event(), torch.cuda.Event()]
     for ev_ in set_free:
         ev_.record(e2e_streams[2])
-    d_host = dataclasses.replace(d, flags=d.flags | dsa.DSA_FLAG_HOST_UNORDERED)
+    # (the host call schedules its own sub-chunks: no L2 sub-blocks there)
+    d_host = dataclasses.replace(d, flags=(d.flags & ~dsa.DSA_FLAG_L2_SCORES) | dsa.DSA_FLAG_HOST_UNORDERED)
     e2e_calls = [0]
 
     def e2e_step(n_sub):
@@ -547,6 +554,7 @@ def run_ours(args):
                    "d_latent": d.d_latent, "d_rope": d.d_rope, "n_idx_heads": d.n_idx_heads,
                    "d_idx": d.d_idx, "parallelism": f"dp{world} (independent chunks)",
                    "indexer": "fp8 (e4m3) variant" if args.fp8_indexer else "bf16",
+                   "scores": "L2-resident query sub-blocks" if args.l2_scores else "whole chunk",
                    "l2": "flushed: 256 MB write between timed steps"},
         "tflops": tflops,
         "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
@@ -780,6 +788,9 @@ def main():
                     help="also time the attention step's other forms (decode split, block union)")
     ap.add_argument("--fp8-indexer", action="store_true",
                     help="the layer with the FP8 indexer variant (dims.flags = DSA_FLAG_FP8_INDEXER)")
+    ap.add_argument("--l2-scores", action="store_true",
+                    help="the layer's indexer and top-k over query sub-blocks whose scores stay in L2 "
+                         "(dims.flags = DSA_FLAG_L2_SCORES)")
     ap.add_argument("--layer-only", action="store_true",
                     help="time the layer alone and print a short line (for profiler captures)")
     args = ap.parse_args()

@@ -81,6 +81,15 @@ typedef struct dsa_dims {
  * the copy-in of one chunk then overlaps the layers and the copy-out of the
  * previous one. The other calls reject it (DSA_ERR_DIMS). */
 #define DSA_FLAG_HOST_UNORDERED 4u
+/* dims.flags: dsa_prefill_layer scores and selects over query sub-blocks
+ * whose float32 scores fit 64 MiB (a multiple of 64 rows, at least 64: 960
+ * rows at a 17,408-token context), one sub-block after the other. The score
+ * matrix then stays in L2 between the indexer that writes it and the top-k
+ * that reads it, instead of making a round trip through HBM. The workspace
+ * (dsa_workspace_size with the same dims) holds one sub-block's scores.
+ * Selections, outputs and lse are bit-identical to the default schedule.
+ * Not with DSA_FLAG_FP8_INDEXER; the other calls reject it (DSA_ERR_DIMS). */
+#define DSA_FLAG_L2_SCORES 8u
 
 /* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):
  *   (n_heads, d_latent, d_rope)  in {(4, 64, 16), (32, 512, 64)}

@@ -49,6 +49,7 @@ DSA_WS_BLOCK_ATTN = 6
 DSA_FLAG_FP8_INDEXER = 1
 DSA_FLAG_ATTN_PAIR = 2
 DSA_FLAG_HOST_UNORDERED = 4
+DSA_FLAG_L2_SCORES = 8
 DSA_MAX_BLOCK_QUERIES = 2
 
 DSA_MAX_TOPK = 2048

@@ -68,8 +68,21 @@ dsa_status check_dims(const dsa_dims* d, bool need_attn, bool need_indexer,
 
 int64_t layer_ld(const dsa_dims& d) { return (static_cast<int64_t>(d.ctx_len) + 127) / 128 * 128; }
 
+bool l2_scores(const dsa_dims& d) { return (d.flags & DSA_FLAG_L2_SCORES) != 0u; }
+
+// DSA_FLAG_L2_SCORES: query rows per sub-block, so that a sub-block's float32
+// scores (rows x ld) take at most 64 MiB of the 126 MB L2 and stay there
+// between the indexer that writes them and the top-k that reads them; a
+// multiple of 64 rows, at least 64
+int l2_subblock_rows(const dsa_dims& d) {
+  const int64_t rows = (static_cast<int64_t>(64) << 20) / (layer_ld(d) * 4);
+  const int64_t r = rows < 64 ? 64 : rows / 64 * 64;
+  return static_cast<int>(r < d.n_q ? r : d.n_q);
+}
+
 size_t layer_scores_bytes(const dsa_dims& d) {
-  return static_cast<size_t>(d.n_q) * layer_ld(d) * sizeof(float);
+  const int64_t rows = l2_scores(d) ? l2_subblock_rows(d) : d.n_q;
+  return static_cast<size_t>(rows) * layer_ld(d) * sizeof(float);
 }
 
 
@@ -195,9 +208,21 @@ dsa_status enqueue_layer(const dsa_dims& d, const uint16_t* q, const uint16_t* l
       e = dsa::launch_key_norm_max(d, k_idx, h, st);
       if (e == cudaSuccess) e = dsa::launch_attn_key_norm_max(d, latent, rope, h, st);
     }
-    if (e == cudaSuccess) e = dsa::launch_index_scores(d, q_idx, k_idx, w_idx, scores, ld, h, st);
-    if (e != cudaSuccess) return DSA_ERR_CUDA;
-    e = dsa::launch_topk(d, scores, ld, q_idx, k_idx, w_idx, idx, h, cand, st);
+    // scores then selection, over the whole chunk or (DSA_FLAG_L2_SCORES)
+    // over query sub-blocks whose scores stay in L2; a row's scores and
+    // selection do not depend on the rows launched with it
+    const int step = l2_scores(d) ? l2_subblock_rows(d) : d.n_q;
+    for (int r0 = 0; r0 < d.n_q && e == cudaSuccess; r0 += step) {
+      dsa_dims ds = d;
+      ds.n_q = d.n_q - r0 < step ? d.n_q - r0 : step;
+      ds.q_pos0 = d.q_pos0 + r0;
+      const uint16_t* qi = q_idx + static_cast<int64_t>(r0) * d.n_idx_heads * d.d_idx;
+      const float* wi = w_idx + static_cast<int64_t>(r0) * d.n_idx_heads;
+      e = dsa::launch_index_scores(ds, qi, k_idx, wi, scores, ld, h, st);
+      if (e == cudaSuccess)
+        e = dsa::launch_topk(ds, scores, ld, qi, k_idx, wi, idx + static_cast<int64_t>(r0) * d.top_k, h,
+                             cand, st);
+    }
   }
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   if (decode) {
@@ -403,8 +428,10 @@ dsa_status dsa_prefill_layer(const dsa_dims* d, const uint16_t* q, const uint16_
                              const uint16_t* rope, const uint16_t* q_idx, const uint16_t* k_idx,
                              const float* w_idx, uint16_t* out, float* lse, int32_t* idx_out,
                              void* ws, size_t ws_bytes, void* stream) {
-  dsa_status s = check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR);
+  dsa_status s =
+      check_dims(d, true, true, DSA_FLAG_FP8_INDEXER | DSA_FLAG_ATTN_PAIR | DSA_FLAG_L2_SCORES);
   if (s != DSA_OK) return s;
+  if (fp8_indexer(*d) && l2_scores(*d)) return DSA_ERR_DIMS;  // sub-blocks: bf16 indexer only
   if (!q || !latent || !rope || !q_idx || !k_idx || !w_idx || !out) return DSA_ERR_NULL;
   if (!aligned16(q) || !aligned16(latent) || !aligned16(rope) || !aligned16(q_idx) ||
       !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(out) || (lse && !aligned16(lse)) ||

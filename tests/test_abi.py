@@ -91,6 +91,26 @@ def test_workspace_sizes(dsa):
             256 + n_q * ldl * 4 + n_q * 2048 * 4 + cand
 
 
+def test_l2_scores_workspace_and_flag_rules(dsa):
+    import dataclasses
+
+    d = workloads.BY_NAME["chunk8k_ctx17k"].dims
+    ld = (d.ctx_len + 127) // 128 * 128
+    rows = (64 << 20) // (ld * 4) // 64 * 64  # 960 rows of 17,408 keys
+    assert rows == 960
+    dl2 = dataclasses.replace(d, flags=dsa.DSA_FLAG_L2_SCORES)
+    assert dsa.dsa_workspace_size(dl2, dsa.DSA_WS_LAYER) == 256 + rows * ld * 4 + d.n_q * d.top_k * 4
+    small = workloads.make_dims(40, 100, 140, 32, 512, 64, 32, 128, 64)  # fewer rows than a sub-block
+    sl2 = dataclasses.replace(small, flags=dsa.DSA_FLAG_L2_SCORES)
+    assert dsa.dsa_workspace_size(sl2, dsa.DSA_WS_LAYER) == dsa.dsa_workspace_size(small, dsa.DSA_WS_LAYER)
+    # not with the FP8 indexer; the calls other than dsa_prefill_layer reject it
+    both = dataclasses.replace(d, flags=dsa.DSA_FLAG_L2_SCORES | dsa.DSA_FLAG_FP8_INDEXER)
+    assert _layer(dsa, both) == dsa.DSA_ERR_DIMS
+    assert dsa.dsa_topk_select(dl2, FAKE, ld, None, None, None, FAKE, FAKE, 1 << 30, 0) == dsa.DSA_ERR_DIMS
+    assert dsa.dsa_decode_layer(dl2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                                1 << 40, stream=0) == dsa.DSA_ERR_DIMS
+
+
 FAKE = 1 << 20  # an aligned, never dereferenced address
 
 

@@ -391,6 +391,26 @@ def test_bounded_wait_gives_up_cleanly(dsa, oracle_lib):
     _compare_layer(oracle_lib, d, x, out, lse, idx)
 
 
+@pytest.mark.parametrize("name,n_rows", [("chunk8k_ctx17k", None), ("chunk4k_ctx128k", 1100)])
+def test_l2_scores_schedule_is_bit_identical(dsa, name, n_rows):
+    """DSA_FLAG_L2_SCORES (indexer and top-k over query sub-blocks whose
+    scores stay in L2): selections, outputs and lse equal the default
+    schedule's bit for bit, on the full 8K chunk (nine sub-blocks) and on rows
+    of the 131,072-token context (two-pass top-k, 128-row sub-blocks)."""
+    import dataclasses
+
+    d, x = workloads.workload_inputs(name)
+    if n_rows is not None:
+        d = dataclasses.replace(d, n_q=n_rows, q_pos0=d.ctx_len - n_rows)
+        x = workloads.generate(d, 5, "normal", "uniform")
+    xd = stage(x)
+    out0, lse0, idx0 = run_layer(dsa, d, xd)
+    out1, lse1, idx1 = run_layer(dsa, dataclasses.replace(d, flags=dsa.DSA_FLAG_L2_SCORES), xd)
+    assert np.array_equal(idx0, idx1)
+    assert np.array_equal(out0, out1)
+    assert np.array_equal(lse0, lse1)
+
+
 def test_mma_layout_selftest_passes(dsa):
     """The start-up check of the tensor-core operand layouts: every accumulator
     element of the four forms (indexer bf16, attention QK^T and PV, FP8
