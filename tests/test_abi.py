@@ -39,6 +39,21 @@ def test_header_declares_the_entry_points():
         assert n in names
 
 
+def test_header_is_plain_c99(tmp_path):
+    """The boundary is a C ABI: include/dsa.h compiles as strict C99."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_dsa.c"
+    src.write_text('#include "dsa.h"\nint main(void) { dsa_dims d = {0}; (void)d; return 0; }\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_library_exports_every_declared_symbol(dsa):
     lib = ctypes.CDLL(dsa.LIB_PATH)
     for name in declared_functions():
