@@ -88,7 +88,9 @@ typedef struct dsa_dims {
  * that reads it, instead of making a round trip through HBM. The workspace
  * (dsa_workspace_size with the same dims) holds one sub-block's scores.
  * Selections, outputs and lse are bit-identical to the default schedule.
- * Not with DSA_FLAG_FP8_INDEXER; the other calls reject it (DSA_ERR_DIMS). */
+ * dsa_prefill_layer_noalloc accepts it too (its scratch then holds the
+ * sub-block workspace). Not with DSA_FLAG_FP8_INDEXER; the other calls reject
+ * it (DSA_ERR_DIMS). */
 #define DSA_FLAG_L2_SCORES 8u
 
 /* Supported shapes (anything else returns DSA_ERR_DIMS; there is no fallback):

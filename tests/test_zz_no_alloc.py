@@ -62,6 +62,22 @@ def test_noalloc_matches_layer_on_two_calls_in_a_row(dsa):
         assert np.array_equal(lse, ref_lse)
 
 
+def test_noalloc_accepts_the_l2_sub_block_schedule(dsa):
+    """DSA_FLAG_L2_SCORES through the call without allocation: the same bits as
+    dsa_prefill_layer with and without the flag (the 157-query chunk is one
+    sub-block, so the schedule and workspace equal the default's)."""
+    import dataclasses
+
+    d, x = _reduced_chunk()
+    xd = stage(x)
+    dl2 = dataclasses.replace(d, flags=dsa.DSA_FLAG_L2_SCORES)
+    out, lse, idx = _noalloc(dsa, dl2, xd)
+    ref_out, ref_lse, ref_idx = run_layer(dsa, d, xd)
+    assert np.array_equal(idx, ref_idx)
+    assert np.array_equal(out, ref_out)
+    assert np.array_equal(lse, ref_lse)
+
+
 def _scratch_bytes(n_q, T, k):
     return 256 + n_q * ((T + 127) // 128 * 128 + k) * 4
 
